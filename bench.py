@@ -1,0 +1,422 @@
+#!/usr/bin/env python
+"""Benchmark: one step = the whole hot path on the 128K last-chunk workload.
+
+Workload (one LLaMA-3.1-8B attention layer, last chunk of a 128K prompt):
+32 query heads / 8 KV heads, head_dim 128, bf16, prefix 129024 + chunk 2048
+tokens, block = page = 64 tokens, randomly permuted pages, vertical-slash
+masks (sink, 8-block local window, 5% columns shared 70% within a group).
+
+Step = ca_build_tables (Q-block + intra-group union, compaction) followed by
+ca_chunk_attention (paged, in place) on device-resident inputs.  Four input
+sets (distinct page buffers and masks) rotate between steps so that a step
+never finds the previous step's selected pages in L2.
+
+value = selected-block FLOPs per step / device time per step (TFLOP/s);
+e2e   = the same metric through the public API with pinned host buffers:
+        H2D of the mask, Q, the chunk's own K/V pages and the page table,
+        build + attention, D2H of O and LSE, all inside the timed region.
+Also reported: the density-100% path on the same shapes (attention speedup),
+the batched table builder in GB/s (32 masks per launch), roofline fractions
+against the measured peaks, and the float64 oracle timed on host cores.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+Under torchrun every rank runs its own replica of the workload (weak scaling,
+no collective on the data path); rank 0 prints one JSON line.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "chunk attn ms & TFLOP/s (selected blocks) vs dense at 128K; table build GB/s"
+WORKLOAD = ("ctx128k: Hq 32 / Hkv 8, d 128, bf16, prefix 129024 + chunk 2048, block 64, "
+            "paged KV with random page permutation, vertical-slash masks (rho_col 0.05, "
+            "corr 0.7, window 8)")
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "samples": len(sm), "power_w_max": max(power) if power else None,
+                "reasons": sorted(reasons)}
+
+
+def make_sets(w, nsets, dev):
+    """nsets input sets on the device: distinct page buffers (same values, distinct
+    addresses) and masks drawn with seeds 0..nsets-1."""
+    import torch
+
+    import workloads
+    x = workloads.make_qkv_pages(w, seed=0)
+    base = {k: v.to(dev) for k, v in x.items()}
+    sets = []
+    for s in range(nsets):
+        m = torch.from_numpy(workloads.mask_for(w, seed=s)).to(dev)
+        d = {"Q": base["Q"].clone(), "K": base["K_pages"].clone(), "V": base["V_pages"].clone(),
+             "pt": base["page_table"].clone(), "mask": m,
+             "tables": torch.empty(w.Hkv, w.nKblk, dtype=torch.int32, device=dev),
+             "counts": torch.empty(w.Hkv, dtype=torch.int32, device=dev),
+             "O": torch.empty_like(base["Q"]),
+             "LSE": torch.empty(w.Hq, w.chunk_len, dtype=torch.float32, device=dev)}
+        sets.append(d)
+    return x, sets
+
+
+def run_step(bsc, w, s, ws, err):
+    bsc.build_tables(s["mask"], w.Hkv, s["tables"], s["counts"])
+    bsc.chunk_attention(s["Q"], s["K"], s["V"], s["pt"], s["tables"], s["counts"],
+                        w.prefix_len, err_flag=err, out=s["O"], lse=s["LSE"], workspace=ws)
+
+
+def cpu_oracle_sample(w, x, mask, budget_s=12.0, stride=None):
+    """Time the float64 oracle (tables in full + attention on a row sample) on host cores."""
+    import numpy as np
+
+    import block_sparse_chunked_b200 as bsc
+    import oracle
+    t0 = time.perf_counter()
+    t, c = oracle.oracle_tables(mask, w.Hkv)
+    t_tab = time.perf_counter() - t0
+    G = w.G
+    live = {}
+    for g in range(w.Hkv):
+        row = t[g, :c[g]]
+        live[g] = np.searchsorted(row, w.nPblk + np.arange(w.nQblk), side="right")
+    # calibrate: a first small sample, then grow the stride-sample to fill the budget
+    Qd = x["Q"].double().numpy()
+    stride = stride or 4
+    rows = [(h, i) for i in range(0, w.chunk_len, stride) for h in range(w.Hq)]
+    t0 = time.perf_counter()
+    oracle.oracle_rows(Qd, x["K_pages"], x["V_pages"], x["page_table"].numpy(), t, c,
+                       w.prefix_len, rows)
+    dt = time.perf_counter() - t0
+    flops = sum(4.0 * w.head_dim * w.block * live[h // G][i // w.block] for h, i in rows)
+    tot_flops = bsc.selected_flops(t, c, w.Hq, w.nPblk, w.nQblk, w.block, w.head_dim)
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:
+        blas = 1
+    return {
+        "value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": int(blas),
+        "host_cpus": len(os.sched_getaffinity(0)), "kind": "oracle",
+        "sample": (f"float64 oracle: tables for the full mask ({t_tab:.2f} s) + attention for "
+                   f"{len(rows)} of {w.Hq * w.chunk_len} query rows (all heads, every "
+                   f"{stride}th token), {flops / 1e9:.1f} of {tot_flops / 1e9:.1f} selected GFLOP, "
+                   f"{dt:.2f} s"),
+        "seconds": dt + t_tab,
+    }
+
+
+def reference_arm(args, rank):
+    """The oracle as the reference implementation, timed on the host cores."""
+    import workloads
+    if rank != 0:
+        return
+    w = workloads.get_config("ctx128k")
+    x = workloads.make_qkv_pages(w, seed=0)
+    mask = workloads.mask_for(w, seed=0)
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, x, mask, stride=256)
+    res = [cpu_oracle_sample(w, x, mask, stride=64) for _ in range(args.steps)]
+    v = statistics.mean(r["value"] for r in res)
+    secs = statistics.mean(r["seconds"] for r in res)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "reference": "float64 CPU oracle (no published code)"},
+        "cpu_baseline": {k: res[-1][k] for k in ("kind", "cores", "sample", "unit")} | {"value": v},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sets", type=int, default=4)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        reference_arm(args, rank)
+        return
+
+    import numpy as np
+    import torch
+
+    import __graft_entry__
+    __graft_entry__.build()
+    import block_sparse_chunked_b200 as bsc
+    import workloads
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    peaks, peak_src = load_peaks()
+    w = workloads.get_config("ctx128k")
+    x, sets = make_sets(w, args.sets, dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws_n = bsc.workspace_size(torch.bfloat16, w.Hq, w.Hkv, w.head_dim, w.block, w.chunk_len,
+                              w.prefix_len, w.num_pages)
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev)
+    launches_per_step = 2 + (1 if ws_n > 0 else 0)
+    stream = torch.cuda.current_stream()
+
+    # ---- warm-up
+    for i in range(args.warmup):
+        run_step(bsc, w, sets[i % len(sets)], ws, err)
+    torch.cuda.synchronize()
+    bsc.check(err)
+
+    # ---- timed region: K steps, per-step events around the builder and the attention
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        s = sets[i % len(sets)]
+        ev[i][0].record(stream)
+        bsc.build_tables(s["mask"], w.Hkv, s["tables"], s["counts"])
+        ev[i][1].record(stream)
+        bsc.chunk_attention(s["Q"], s["K"], s["V"], s["pt"], s["tables"], s["counts"],
+                            w.prefix_len, err_flag=err, out=s["O"], lse=s["LSE"], workspace=ws)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    clk = clocks.stop()
+    bsc.check(err)
+    step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    build_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
+    attn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    flops = []
+    for i in range(args.steps):
+        s = sets[i % len(sets)]
+        flops.append(bsc.selected_flops(s["tables"].cpu().numpy(), s["counts"].cpu().numpy(),
+                                        w.Hq, w.nPblk, w.nQblk, w.block, w.head_dim))
+    mean_step = statistics.mean(step_ms)
+    mean_attn = statistics.mean(attn_ms)
+    mean_flops = statistics.mean(flops)
+    tot = torch.tensor([mean_step, mean_attn], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(tot, op=pg.ReduceOp.MAX)
+    mean_step, mean_attn = float(tot[0]), float(tot[1])
+    value = world * mean_flops / (mean_step * 1e-3) / 1e12
+    attn_tflops = mean_flops / (mean_attn * 1e-3) / 1e12
+
+    # ---- density-100% path on the same shapes (all blocks selected)
+    dense_t = torch.arange(w.nKblk, dtype=torch.int32, device=dev).repeat(w.Hkv, 1).contiguous()
+    dense_c = torch.full((w.Hkv,), w.nKblk, dtype=torch.int32, device=dev)
+    dense_ms = []
+    for i in range(2 + 4):
+        s = sets[i % len(sets)]
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        bsc.chunk_attention(s["Q"], s["K"], s["V"], s["pt"], dense_t, dense_c, w.prefix_len,
+                            err_flag=err, out=s["O"], lse=s["LSE"], workspace=ws)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= 2:
+            dense_ms.append(a.elapsed_time(b))
+    bsc.check(err)
+    dense_flops = bsc.dense_flops(w.Hq, w.nPblk, w.nQblk, w.block, w.head_dim)
+    dense_ms_mean = statistics.mean(dense_ms)
+
+    # ---- batched table builder: 32 masks per launch (one per layer), 4 rotating batches
+    nb = 32
+    import workloads as wl
+    mb = [torch.from_numpy(np.stack([wl.mask_for(w, seed=100 + 32 * r + k) for k in range(nb)]))
+          .to(dev) for r in range(4)]
+    tb = torch.empty(nb, w.Hkv, w.nKblk, dtype=torch.int32, device=dev)
+    cb = torch.empty(nb, w.Hkv, dtype=torch.int32, device=dev)
+    for r in range(4):
+        bsc.build_tables_batched(mb[r], w.Hkv, tb, cb)
+    bt = []
+    for r in range(12):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        bsc.build_tables_batched(mb[r % 4], w.Hkv, tb, cb)
+        b.record(stream)
+        torch.cuda.synchronize()
+        bt.append(a.elapsed_time(b))
+    bbytes = bsc.builder_bytes(nb, w.Hq, w.Hkv, w.nQblk, w.nKblk)
+    build_gbs = bbytes / (statistics.mean(bt) * 1e-3) / 1e9
+    single_bytes = bsc.builder_bytes(1, w.Hq, w.Hkv, w.nQblk, w.nKblk)
+
+    # ---- end to end through the public API with pinned host buffers
+    chunk_blocks = list(range(w.nPblk, w.nKblk))
+    h_mask = torch.from_numpy(wl.mask_for(w, seed=0)).pin_memory()
+    h_q = x["Q"].pin_memory()
+    h_pt = x["page_table"].pin_memory()
+    pt_np = x["page_table"].numpy()
+    h_kc = x["K_pages"][torch.from_numpy(pt_np[chunk_blocks]).long()].contiguous().pin_memory()
+    h_vc = x["V_pages"][torch.from_numpy(pt_np[chunk_blocks]).long()].contiguous().pin_memory()
+    h_o = torch.empty(w.chunk_len, w.Hq, w.head_dim, dtype=torch.bfloat16).pin_memory()
+    h_l = torch.empty(w.Hq, w.chunk_len, dtype=torch.float32).pin_memory()
+    h2d = (h_mask.numel() + h_q.numel() * 2 + h_pt.numel() * 4 + h_kc.numel() * 2 * 2)
+    d2h = h_o.numel() * 2 + h_l.numel() * 4
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        s = sets[i % len(sets)]
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        s["mask"].copy_(h_mask, non_blocking=True)
+        s["Q"].copy_(h_q, non_blocking=True)
+        s["pt"].copy_(h_pt, non_blocking=True)
+        for j, kb in enumerate(chunk_blocks):
+            page = int(pt_np[kb])
+            s["K"][page].copy_(h_kc[j], non_blocking=True)
+            s["V"][page].copy_(h_vc[j], non_blocking=True)
+        bsc.build_tables(s["mask"], w.Hkv, s["tables"], s["counts"])
+        bsc.chunk_attention(s["Q"], s["K"], s["V"], s["pt"], s["tables"], s["counts"],
+                            w.prefix_len, err_flag=err, out=s["O"], lse=s["LSE"], workspace=ws)
+        h_o.copy_(s["O"], non_blocking=True)
+        h_l.copy_(s["LSE"], non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    bsc.check(err)
+    e2e_flops = bsc.selected_flops(sets[0]["tables"].cpu().numpy(),
+                                   sets[0]["counts"].cpu().numpy(), w.Hq, w.nPblk, w.nQblk,
+                                   w.block, w.head_dim)
+    e2e_t = torch.tensor([statistics.mean(e2e_ms)], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(e2e_t, op=pg.ReduceOp.MAX)
+    e2e_value = world * e2e_flops / (float(e2e_t[0]) * 1e-3) / 1e12
+
+    if rank == 0:
+        peak = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
+        peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK["bf16_tflops_sustained"])
+        hbm = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) Q/K/V, vertical-slash masks)",
+            "config": {"workload": WORKLOAD, "parallelism": f"replicas x{world}",
+                       "l2": f"{len(sets)} rotating input sets (distinct page buffers and masks)",
+                       "selected_gflop_per_step": mean_flops / 1e9,
+                       "table_density": float(np.mean([
+                           s["counts"].float().mean().item() / w.nKblk for s in sets]))},
+            "attention_ms": mean_attn, "attention_tflops": attn_tflops,
+            "table_build_us": statistics.mean(build_ms) * 1e3,
+            "table_build_single_gbs": single_bytes / (statistics.mean(build_ms) * 1e-3) / 1e9,
+            "dense_ms": dense_ms_mean, "dense_tflops": dense_flops / (dense_ms_mean * 1e-3) / 1e12,
+            "speedup_vs_dense": dense_ms_mean / mean_attn,
+            "table_build_batched": {"masks_per_launch": nb, "us": statistics.mean(bt) * 1e3,
+                                    "GB/s": build_gbs, "frac_of_measured_hbm": build_gbs / hbm,
+                                    "frac_of_8TBs_nominal": build_gbs / 8000.0},
+            "roofline": {"bound": "tensor", "kernel": "chunk_attn_kernel",
+                         "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": attn_tflops / peak, "peak_source": f"{peak_src} bf16 burst",
+                         "frac_of_sustained": attn_tflops / peak_sus,
+                         "per_launch": "selected FLOPs of one 2048-token chunk (32 heads)",
+                         "traffic": None},
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
+                    "d2h_bytes_per_step": int(d2h), "ms_per_step": float(e2e_t[0])},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            cb_ = cpu_oracle_sample(w, x, wl.mask_for(w, seed=0))
+            cb_.pop("seconds", None)
+            line["cpu_baseline"] = cb_
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,177 @@
+"""ctypes declarations of libcompactattn.so and tensor marshalling."""
+import ctypes
+import os
+
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libcompactattn.so")
+
+CA_OK = 0
+CA_ERR_ARG = -1
+CA_ERR_ALIGN = -2
+CA_ERR_DTYPE = -3
+CA_ERR_LAUNCH = -4
+CA_ERR_BOUNDS = -5
+CA_ERR_TIMEOUT = -6
+CA_ERR_WORKSPACE = -7
+CA_DTYPE_BF16 = 0
+CA_DTYPE_FP32 = 1
+
+_c_int, _c_size, _vp = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+
+# name -> (restype, argtypes); every symbol include/compactattn.h declares
+EXPORTS = {
+    "ca_build_tables": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
+    "ca_build_tables_batched": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp,
+                                         _vp]),
+    "ca_workspace_size": (_c_size, [_c_int] * 9),
+    "ca_chunk_attention": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _vp, _c_int, _c_int,
+                                    _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_size,
+                                    _c_int, _vp, _vp]),
+    "ca_check": (_c_int, [_vp, _vp]),
+    "ca_wait_probe": (_c_int, [_vp, _c_int, _vp]),
+    "ca_last_error": (_c_int, [ctypes.c_char_p, _c_size]),
+    "ca_version": (_c_int, []),
+}
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is not built; run `python block_sparse_chunked_b200/_build.py` "
+            "(nvcc, sm_100a). There is no fallback implementation.")
+    L = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in EXPORTS.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L
+
+
+lib = _load()
+
+
+class CompactAttnError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"[{code}] {msg}")
+        self.code = code
+
+
+def last_error():
+    buf = ctypes.create_string_buffer(1024)
+    lib.ca_last_error(buf, 1024)
+    return buf.value.decode(errors="replace")
+
+
+def _ok(rc):
+    if rc != CA_OK:
+        raise CompactAttnError(rc, last_error())
+
+
+def version():
+    return lib.ca_version()
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _need_cuda(name, t, dtypes=None, ndim=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+
+
+def build_tables_batched(masks, Hkv, tables=None, counts=None):
+    """masks uint8/bool [nb, Hq, nQblk, nKblk] -> tables int32 [nb, Hkv, nKblk], counts [nb, Hkv]."""
+    _need_cuda("masks", masks, (torch.uint8, torch.bool), 4)
+    nb, Hq, nQ, nK = masks.shape
+    if tables is None:
+        tables = torch.empty(nb, Hkv, nK, dtype=torch.int32, device=masks.device)
+    if counts is None:
+        counts = torch.empty(nb, Hkv, dtype=torch.int32, device=masks.device)
+    _ok(lib.ca_build_tables_batched(_ptr(masks), nb, Hq, Hkv, nQ, nK, _ptr(tables), _ptr(counts),
+                                    _stream()))
+    return tables, counts
+
+
+def build_tables(mask, Hkv, tables=None, counts=None):
+    """mask uint8/bool [Hq, nQblk, nKblk] -> (tables int32 [Hkv, nKblk], counts int32 [Hkv])."""
+    _need_cuda("mask", mask, (torch.uint8, torch.bool), 3)
+    Hq, nQ, nK = mask.shape
+    if tables is None:
+        tables = torch.empty(Hkv, nK, dtype=torch.int32, device=mask.device)
+    if counts is None:
+        counts = torch.empty(Hkv, dtype=torch.int32, device=mask.device)
+    _ok(lib.ca_build_tables(_ptr(mask), Hq, Hkv, nQ, nK, _ptr(tables), _ptr(counts), _stream()))
+    return tables, counts
+
+
+_DT = {torch.bfloat16: CA_DTYPE_BF16, torch.float32: CA_DTYPE_FP32}
+
+
+def workspace_size(dtype, Hq, Hkv, head_dim, block, chunk_len, prefix_len, num_pages, n_splits=0):
+    code = _DT[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    n = lib.ca_workspace_size(code, Hq, Hkv, head_dim, block, chunk_len, prefix_len, num_pages,
+                              n_splits)
+    if n == ctypes.c_size_t(-1).value:
+        raise CompactAttnError(CA_ERR_ARG, "invalid shapes for ca_workspace_size")
+    return n
+
+
+def chunk_attention(Q, K_pages, V_pages, page_table, tables, counts, prefix_len, n_splits=0,
+                    err_flag=None, out=None, lse=None, workspace=None):
+    """Chunk attention over the group tables' blocks of a paged KV cache.
+
+    Q [L, Hq, d]; K_pages/V_pages [num_pages, Hkv, B, d] (bf16 or fp32, same
+    dtype); page_table int32 [nKblk]; tables int32 [Hkv, nKblk]; counts int32
+    [Hkv].  Returns O [L, Hq, d] (dtype of Q) and LSE float32 [Hq, L].
+    """
+    _need_cuda("Q", Q, tuple(_DT), 3)
+    _need_cuda("K_pages", K_pages, (Q.dtype,), 4)
+    _need_cuda("V_pages", V_pages, (Q.dtype,), 4)
+    _need_cuda("page_table", page_table, (torch.int32,), 1)
+    _need_cuda("tables", tables, (torch.int32,), 2)
+    _need_cuda("counts", counts, (torch.int32,), 1)
+    if K_pages.shape != V_pages.shape:
+        raise ValueError("K_pages and V_pages must have the same shape")
+    L, Hq, d = Q.shape
+    num_pages, Hkv, B, d2 = K_pages.shape
+    if d2 != d:
+        raise ValueError("head_dim of Q and of the pages differ")
+    nK = (prefix_len + L) // B if B else 0
+    if page_table.numel() < nK or tables.shape[0] != Hkv or tables.shape[1] < nK \
+            or counts.numel() < Hkv:
+        raise ValueError("page_table / tables / counts are smaller than the chunk needs")
+    code = _DT[Q.dtype]
+    if out is None:
+        out = torch.empty_like(Q)
+    if lse is None:
+        lse = torch.empty(Hq, L, dtype=torch.float32, device=Q.device)
+    ws_n = workspace_size(code, Hq, Hkv, d, B, L, prefix_len, num_pages, n_splits)
+    if ws_n and (workspace is None or workspace.numel() < ws_n):
+        workspace = torch.empty(ws_n, dtype=torch.uint8, device=Q.device)
+    _ok(lib.ca_chunk_attention(
+        _ptr(Q), _ptr(K_pages), _ptr(V_pages), code, num_pages, _ptr(page_table), _ptr(tables),
+        _ptr(counts), Hq, Hkv, d, B, L, prefix_len, _ptr(out), _ptr(lse),
+        _ptr(workspace) if ws_n else None, ws_n, n_splits, _ptr(err_flag), _stream()))
+    return out, lse
+
+
+def check(err_flag):
+    """Synchronise, read and clear the device error word; raise on a device error."""
+    _ok(lib.ca_check(_ptr(err_flag), _stream()))
+
+
+def wait_probe(err_flag, limit_us):
+    _ok(lib.ca_wait_probe(_ptr(err_flag), int(limit_us), _stream()))

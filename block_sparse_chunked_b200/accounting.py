@@ -1,0 +1,40 @@
+"""Work and traffic accounting for throughput reporting (host side, numpy).
+
+FLOPs count 4 * B^2 * d per live (query head, Q-block, KV block) pair: two
+B x B x d contractions (Q K^T and P V) at 2 FLOPs per multiply-add.  A pair
+is live when the KV block can hold a key visible to the Q-block
+(kb <= nPblk + qb); diagonal blocks are counted in full.  "Selected" keeps
+only the pairs whose KV block is in the group's table.
+"""
+import numpy as np
+
+
+def selected_pairs(tables, counts, Hq, nPblk, nQblk):
+    tables = np.asarray(tables)
+    counts = np.asarray(counts)
+    Hkv = tables.shape[0]
+    G = Hq // Hkv
+    total = 0
+    diag = nPblk + np.arange(nQblk)
+    for g in range(Hkv):
+        row = np.sort(tables[g, :int(counts[g])])
+        live = np.searchsorted(row, diag, side="right")  # entries <= diagonal, per Q-block
+        total += G * int(live.sum())
+    return total
+
+
+def dense_pairs(Hq, nPblk, nQblk):
+    return Hq * int(sum(nPblk + qb + 1 for qb in range(nQblk)))
+
+
+def selected_flops(tables, counts, Hq, nPblk, nQblk, block, head_dim):
+    return 4.0 * block * block * head_dim * selected_pairs(tables, counts, Hq, nPblk, nQblk)
+
+
+def dense_flops(Hq, nPblk, nQblk, block, head_dim):
+    return 4.0 * block * block * head_dim * dense_pairs(Hq, nPblk, nQblk)
+
+
+def builder_bytes(nb, Hq, Hkv, nQblk, nKblk):
+    """Algorithmic bytes of one table-builder launch: mask read + tables + counts written."""
+    return nb * (Hq * nQblk * nKblk + Hkv * nKblk * 4 + Hkv * 4)

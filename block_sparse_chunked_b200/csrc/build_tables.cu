@@ -1,0 +1,215 @@
+// build_tables.cu — Block-Union KV selection on the GPU.
+//
+// "CompactAttention: Accelerating Chunked Prefill with Block-Union KV
+// Selection", Abstract: the 2D block-sparse masks are turned into GQA-aware
+// per-group KV block tables by a Q-block union and an intra-group union, the
+// minimal tables that keep every selected block.
+//
+// The rows of one group (G heads x nQblk Q-blocks) are contiguous in the mask,
+// so the union is an OR-reduction of an [G*nQblk, nKblk] byte matrix down its
+// rows, and the table is the ordered list of nonzero columns.  One thread
+// block cluster (up to 8 CTAs) owns one (mask, group): each CTA reduces a
+// column slab with 16-, 4- or 1-byte loads, turns it into a bit set in shared
+// memory, and compacts it with per-word popcounts and a block scan; the CTAs
+// exchange their slab counts through distributed shared memory to place
+// their entries.  No global scratch, no atomics on global memory, and the
+// output is deterministic.  HBM-bound: every mask byte is read exactly once.
+#include <cooperative_groups.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace ca {
+
+constexpr int kBuildThreads = 256;
+constexpr int kMaxSlab = 8192;  // columns per CTA -> 256 bit-set words, one per thread
+
+template <int VEC>
+struct VecLoad;
+template <>
+struct VecLoad<16> {
+  using T = uint4;
+  __device__ static uint4 zero() { return make_uint4(0, 0, 0, 0); }
+  __device__ static void orin(uint4& a, const uint4& b) {
+    a.x |= b.x; a.y |= b.y; a.z |= b.z; a.w |= b.w;
+  }
+  // byte i of the 16 -> bit i
+  __device__ static uint32_t bits(const uint4& a) {
+    auto nb = [](uint32_t x) {
+      uint32_t m = __vcmpne4(x, 0u);  // 0xFF in each nonzero byte
+      return ((m >> 7) & 1u) | ((m >> 14) & 2u) | ((m >> 21) & 4u) | ((m >> 28) & 8u);
+    };
+    return nb(a.x) | (nb(a.y) << 4) | (nb(a.z) << 8) | (nb(a.w) << 12);
+  }
+};
+template <>
+struct VecLoad<4> {
+  using T = uint32_t;
+  __device__ static uint32_t zero() { return 0u; }
+  __device__ static void orin(uint32_t& a, const uint32_t& b) { a |= b; }
+  __device__ static uint32_t bits(const uint32_t& a) {
+    uint32_t m = __vcmpne4(a, 0u);
+    return ((m >> 7) & 1u) | ((m >> 14) & 2u) | ((m >> 21) & 4u) | ((m >> 28) & 8u);
+  }
+};
+template <>
+struct VecLoad<1> {
+  using T = uint8_t;
+  __device__ static uint8_t zero() { return 0; }
+  __device__ static void orin(uint8_t& a, const uint8_t& b) { a |= b; }
+  __device__ static uint32_t bits(const uint8_t& a) { return a != 0; }
+};
+
+// grid = (C, Hkv, nb), cluster = (C, 1, 1); slab = columns per CTA (multiple of 32).
+template <int VEC>
+__global__ void __launch_bounds__(kBuildThreads)
+    build_tables_kernel(const uint8_t* __restrict__ mask, int Hq, int Hkv, int nQblk, int nKblk,
+                        int slab, int32_t* __restrict__ tables, int32_t* __restrict__ counts) {
+  using V = VecLoad<VEC>;
+  using T = typename V::T;
+  __shared__ uint32_t bits[kMaxSlab / 32];
+  __shared__ int warp_sum[kBuildThreads / 32];
+  __shared__ int slab_total;
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int C = (int)cluster.num_blocks();
+  const int tid = threadIdx.x;
+  const int g = blockIdx.y;
+  const int b = blockIdx.z;
+  const int G = Hq / Hkv;
+  const int R = G * nQblk;  // rows of this group
+
+  const uint8_t* base = mask + ((size_t)b * Hq + (size_t)g * G) * (size_t)nQblk * nKblk;
+  const int c0 = rank * slab;
+  const int c1 = min(nKblk, c0 + slab);
+  const int ncols = max(0, c1 - c0);
+  const int nwords = (ncols + 31) >> 5;
+
+  for (int w = tid; w < kMaxSlab / 32; w += kBuildThreads) bits[w] = 0u;
+  __syncthreads();
+
+  // ---- Q-block union + intra-group union: OR down the group's rows.
+  const int ncv = ncols / VEC;  // nKblk % VEC == 0 and c0 % VEC == 0
+  int CW = 1;
+  while (CW < ncv && CW < kBuildThreads) CW <<= 1;
+  const int RT = kBuildThreads / CW;
+  const int rt = tid / CW;
+  for (int v = tid % CW; v < ncv; v += CW) {
+    T acc = V::zero();
+    if (rt < R) {
+      const T* p = reinterpret_cast<const T*>(base + (size_t)rt * nKblk + c0) + v;
+      const size_t step = (size_t)RT * nKblk / VEC;
+      int r = rt;
+#pragma unroll 8
+      for (; r < R; r += RT) {
+        V::orin(acc, __ldg(p));
+        p += step;
+      }
+    }
+    uint32_t m = V::bits(acc);
+    if (m) {
+      const int col = v * VEC;  // within slab
+      atomicOr(&bits[col >> 5], m << (col & 31));
+    }
+  }
+  __syncthreads();
+
+  // ---- compaction: popcount per 32-column word, exclusive block scan.
+  const int lane = tid & 31, warp = tid >> 5;
+  uint32_t word = (tid < nwords) ? bits[tid] : 0u;
+  int cnt = __popc(word);
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sum[warp] = incl;
+  __syncthreads();
+  int wbase = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kBuildThreads / 32; ++w) {
+    wbase += (w < warp) ? warp_sum[w] : 0;
+    tot += warp_sum[w];
+  }
+  const int excl = wbase + incl - cnt;
+  if (tid == 0) slab_total = tot;
+
+  // ---- cluster: offsets of this slab and the group's total through DSMEM.
+  cluster.sync();
+  int before = 0, total = 0;
+  for (int r = 0; r < C; ++r) {
+    const int t = *cluster.map_shared_rank(&slab_total, r);
+    before += (r < rank) ? t : 0;
+    total += t;
+  }
+
+  int32_t* trow = tables + ((size_t)b * Hkv + g) * nKblk;
+  // Each warp writes the entries of its 32 words: for word j, lane l handles
+  // column 32j+l; its position is the word's offset plus the set bits below l.
+  for (int j = 0; j < 32; ++j) {
+    const uint32_t wj = __shfl_sync(0xffffffffu, word, j);
+    const int oj = __shfl_sync(0xffffffffu, excl, j);
+    if (wj == 0u) continue;
+    if ((wj >> lane) & 1u) {
+      const int pos = before + oj + __popc(wj & ((1u << lane) - 1u));
+      trow[pos] = c0 + (warp * 32 + j) * 32 + lane;
+    }
+  }
+  // -1 padding of the positions [total, nKblk) that fall inside this slab.
+  for (int p = max(total, c0) + tid; p < c1; p += kBuildThreads) trow[p] = -1;
+  if (rank == 0 && tid == 0) counts[(size_t)b * Hkv + g] = total;
+  cluster.sync();  // keep slab_total alive until every CTA has read it
+}
+
+template __global__ void build_tables_kernel<16>(const uint8_t*, int, int, int, int, int,
+                                                 int32_t*, int32_t*);
+template __global__ void build_tables_kernel<4>(const uint8_t*, int, int, int, int, int, int32_t*,
+                                                int32_t*);
+template __global__ void build_tables_kernel<1>(const uint8_t*, int, int, int, int, int, int32_t*,
+                                                int32_t*);
+
+// Host launcher: picks the vector width and the cluster size.
+cudaError_t launch_build_tables(const uint8_t* mask, int nb, int Hq, int Hkv, int nQblk,
+                                int nKblk, int32_t* tables, int32_t* counts,
+                                cudaStream_t stream) {
+  int C = (nKblk + 255) / 256;  // ~256+ columns per CTA
+  if (C > 8) C = 8;
+  if (C < 1) C = 1;
+  int slab = (nKblk + C - 1) / C;
+  slab = (slab + 31) & ~31;
+  if (slab > kMaxSlab) return cudaErrorInvalidValue;  // nKblk > 65536
+  C = (nKblk + slab - 1) / slab;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(mask);
+  int vec = 1;
+  if (nKblk % 16 == 0 && a % 16 == 0) vec = 16;
+  else if (nKblk % 4 == 0 && a % 4 == 0) vec = 4;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(C, Hkv, nb);
+  cfg.blockDim = dim3(kBuildThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (vec == 16)
+    return cudaLaunchKernelEx(&cfg, build_tables_kernel<16>, mask, Hq, Hkv, nQblk, nKblk, slab,
+                              tables, counts);
+  if (vec == 4)
+    return cudaLaunchKernelEx(&cfg, build_tables_kernel<4>, mask, Hq, Hkv, nQblk, nKblk, slab,
+                              tables, counts);
+  return cudaLaunchKernelEx(&cfg, build_tables_kernel<1>, mask, Hq, Hkv, nQblk, nKblk, slab,
+                            tables, counts);
+}
+
+}  // namespace ca

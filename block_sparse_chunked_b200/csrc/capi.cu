@@ -1,0 +1,316 @@
+// capi.cu — the extern "C" boundary of libcompactattn.so: argument checks,
+// TMA tensor maps over the paged KV cache, work/split planning, launches and
+// error reporting.  The call signatures are declared and documented in
+// include/compactattn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "compactattn.h"
+#include "internal.h"
+
+namespace ca {
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(CA_ERR_LAUNCH, "%s: %s", what, cudaGetErrorString(e));
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encoder() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+constexpr int kSMs = 148;
+constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per pipeline wait
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Plan {
+  int G, HPU, NT, nhalves, nqs, nPblk, nKblk, spb, n_splits;
+};
+
+bool plan(int Hq, int Hkv, int head_dim, int block, int chunk_len, int prefix_len, int n_splits,
+          Plan& pl) {
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return false;
+  if (head_dim != 64 && head_dim != 128) return false;
+  if (block != 64 && block != 128) return false;
+  if (chunk_len < 64 || prefix_len < 0) return false;
+  if (chunk_len % block || prefix_len % block) return false;
+  pl.G = Hq / Hkv;
+  pl.HPU = pl.G < 4 ? pl.G : 4;
+  pl.NT = (pl.HPU + 1) / 2;
+  pl.nhalves = (pl.G + pl.HPU - 1) / pl.HPU;
+  pl.nqs = chunk_len / 64;
+  pl.nPblk = prefix_len / block;
+  pl.nKblk = (prefix_len + chunk_len) / block;
+  pl.spb = 128 / block;
+  const long long units = (long long)Hkv * pl.nhalves * pl.nqs;
+  const int max_stages = (pl.nKblk + pl.spb - 1) / pl.spb;
+  int S = n_splits;
+  if (S <= 0) {
+    S = 1;
+    if (units < kSMs) S = (int)((2 * kSMs + units - 1) / units);
+    if (S > 16) S = 16;
+  }
+  if (S > max_stages) S = max_stages;
+  if (S < 1) S = 1;
+  if (units * S > 0x7fffffffLL) return false;
+  pl.n_splits = S;
+  return true;
+}
+
+struct WsLayout {
+  size_t opart = 0, lsepart = 0, q = 0, qlo = 0, k = 0, v = 0, total = 0;
+};
+
+WsLayout ws_layout(int dtype, int Hq, int Hkv, int D, int B, int L, int num_pages, int S) {
+  WsLayout w;
+  size_t off = 0;
+  if (S > 1) {
+    w.opart = off;
+    off = align256(off + (size_t)S * L * Hq * D * 4);
+    w.lsepart = off;
+    off = align256(off + (size_t)S * Hq * L * 4);
+  }
+  if (dtype == CA_DTYPE_FP32) {
+    w.q = off;
+    off = align256(off + (size_t)L * Hq * D * 2);
+    w.qlo = off;
+    off = align256(off + (size_t)L * Hq * D * 2);
+    w.k = off;
+    off = align256(off + (size_t)num_pages * Hkv * B * D * 2);
+    w.v = off;
+    off = align256(off + (size_t)num_pages * Hkv * B * D * 2);
+  }
+  w.total = off;
+  return w;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace ca
+
+using namespace ca;
+
+extern "C" {
+
+int ca_version(void) { return 100; }
+
+int ca_last_error(char* buf, size_t n) {
+  if (!buf || n == 0) return CA_ERR_ARG;
+  const size_t m = g_last_error.size() < n - 1 ? g_last_error.size() : n - 1;
+  memcpy(buf, g_last_error.data(), m);
+  buf[m] = 0;
+  return CA_OK;
+}
+
+int ca_build_tables_batched(const uint8_t* masks, int nb, int Hq, int Hkv, int nQblk, int nKblk,
+                            int32_t* tables, int32_t* counts, void* stream) {
+  if (!masks || !tables || !counts) return fail(CA_ERR_ARG, "ca_build_tables: null pointer");
+  if (nb < 1 || nb > 65535) return fail(CA_ERR_ARG, "ca_build_tables: nb=%d out of [1,65535]", nb);
+  if (Hq < 1 || Hkv < 1 || Hkv > Hq || Hq % Hkv)
+    return fail(CA_ERR_ARG, "ca_build_tables: Hq=%d must be a positive multiple of Hkv=%d", Hq, Hkv);
+  if (Hkv > 65535) return fail(CA_ERR_ARG, "ca_build_tables: Hkv=%d too large", Hkv);
+  if (nQblk < 1) return fail(CA_ERR_ARG, "ca_build_tables: nQblk=%d < 1", nQblk);
+  if (nKblk < 1 || nKblk > 65536)
+    return fail(CA_ERR_ARG, "ca_build_tables: nKblk=%d out of [1,65536]", nKblk);
+  cudaError_t e = launch_build_tables(masks, nb, Hq, Hkv, nQblk, nKblk, tables, counts,
+                                      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "ca_build_tables launch");
+  return CA_OK;
+}
+
+int ca_build_tables(const uint8_t* mask, int Hq, int Hkv, int nQblk, int nKblk, int32_t* tables,
+                    int32_t* counts, void* stream) {
+  return ca_build_tables_batched(mask, 1, Hq, Hkv, nQblk, nKblk, tables, counts, stream);
+}
+
+size_t ca_workspace_size(int dtype, int Hq, int Hkv, int head_dim, int block, int chunk_len,
+                         int prefix_len, int num_pages, int n_splits) {
+  Plan pl;
+  if (dtype != CA_DTYPE_BF16 && dtype != CA_DTYPE_FP32) return (size_t)-1;
+  if (!plan(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl)) return (size_t)-1;
+  if (num_pages < pl.nKblk) return (size_t)-1;
+  return ws_layout(dtype, Hq, Hkv, head_dim, block, chunk_len, num_pages, pl.n_splits).total;
+}
+
+int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, int dtype,
+                       int num_pages, const int32_t* page_table, const int32_t* tables,
+                       const int32_t* counts, int Hq, int Hkv, int head_dim, int block,
+                       int chunk_len, int prefix_len, void* O, float* LSE, void* workspace,
+                       size_t ws_bytes, int n_splits, int32_t* err_flag, void* stream) {
+  if (!Q || !K_pages || !V_pages || !page_table || !tables || !counts || !O || !LSE)
+    return fail(CA_ERR_ARG, "ca_chunk_attention: null pointer");
+  if (dtype != CA_DTYPE_BF16 && dtype != CA_DTYPE_FP32)
+    return fail(CA_ERR_DTYPE, "ca_chunk_attention: dtype code %d not supported", dtype);
+  if (block != 64 && block != 128)
+    return fail(CA_ERR_ARG, "ca_chunk_attention: block=%d must be 64 or 128", block);
+  if (chunk_len % block || prefix_len % block)
+    return fail(CA_ERR_ALIGN,
+                "ca_chunk_attention: prefix_len=%d and chunk_len=%d must be multiples of block=%d",
+                prefix_len, chunk_len, block);
+  Plan pl;
+  if (!plan(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl))
+    return fail(CA_ERR_ARG,
+                "ca_chunk_attention: unsupported shape Hq=%d Hkv=%d head_dim=%d block=%d "
+                "chunk_len=%d prefix_len=%d",
+                Hq, Hkv, head_dim, block, chunk_len, prefix_len);
+  if (num_pages < pl.nKblk)
+    return fail(CA_ERR_ARG, "ca_chunk_attention: num_pages=%d < nKblk=%d", num_pages, pl.nKblk);
+  if (!aligned16(Q) || !aligned16(K_pages) || !aligned16(V_pages) || !aligned16(O))
+    return fail(CA_ERR_ARG, "ca_chunk_attention: Q, K_pages, V_pages and O must be 16-byte aligned");
+  const WsLayout wl =
+      ws_layout(dtype, Hq, Hkv, head_dim, block, chunk_len, num_pages, pl.n_splits);
+  if (wl.total > 0 && (!workspace || ws_bytes < wl.total || !aligned16(workspace)))
+    return fail(CA_ERR_WORKSPACE, "ca_chunk_attention: workspace of %zu bytes needed, got %zu",
+                wl.total, workspace ? ws_bytes : (size_t)0);
+  EncodeTiledFn enc = encoder();
+  if (!enc) return fail(CA_ERR_LAUNCH, "ca_chunk_attention: cuTensorMapEncodeTiled unavailable");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int D = head_dim, B = block, L = chunk_len;
+
+  const void* q = Q;
+  const void* qlo = Q;
+  const void* kp = K_pages;
+  const void* vp = V_pages;
+  cudaError_t e;
+  if (dtype == CA_DTYPE_FP32) {
+    // The tensor-core path is bf16 in, fp32 accumulate.  Q is kept as two
+    // bf16 terms (its rounding error would shift every score of a row the
+    // same way); K and V are rounded once.
+    e = launch_split_f32_bf16(static_cast<const float*>(Q), ws + wl.q, ws + wl.qlo,
+                              (size_t)L * Hq * D, st);
+    if (e == cudaSuccess)
+      e = launch_cast_f32_bf16(static_cast<const float*>(K_pages), ws + wl.k,
+                               (size_t)num_pages * Hkv * B * D, st);
+    if (e == cudaSuccess)
+      e = launch_cast_f32_bf16(static_cast<const float*>(V_pages), ws + wl.v,
+                               (size_t)num_pages * Hkv * B * D, st);
+    if (e != cudaSuccess) return cuda_fail(e, "ca_chunk_attention cast");
+    q = ws + wl.q;
+    qlo = ws + wl.qlo;
+    kp = ws + wl.k;
+    vp = ws + wl.v;
+  }
+
+  CUtensorMap tq, tqlo, tk, tv;
+  for (int which = 0; which < 2; ++which) {
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)L};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+    cuuint32_t box[3] = {64, 1, 64};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = enc(which ? &tqlo : &tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                     const_cast<void*>(which ? qlo : q), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(CA_ERR_LAUNCH, "tensor map (Q) encode failed: %d", (int)r);
+  }
+  for (int which = 0; which < 2; ++which) {
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)B, (cuuint64_t)Hkv, (cuuint64_t)num_pages};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)B * D * 2,
+                             (cuuint64_t)Hkv * B * D * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)B, 1, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = enc(which ? &tv : &tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                     const_cast<void*>(which ? vp : kp), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+      return fail(CA_ERR_LAUNCH, "tensor map (%s pages) encode failed: %d", which ? "V" : "K",
+                  (int)r);
+  }
+
+  AttnParams p;
+  p.page_table = page_table;
+  p.tables = tables;
+  p.counts = counts;
+  p.O = O;
+  p.LSE = LSE;
+  p.Opart = pl.n_splits > 1 ? reinterpret_cast<float*>(ws + wl.opart) : nullptr;
+  p.LSEpart = pl.n_splits > 1 ? reinterpret_cast<float*>(ws + wl.lsepart) : nullptr;
+  p.err = err_flag;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = pl.G;
+  p.HPU = pl.HPU;
+  p.nhalves = pl.nhalves;
+  p.L = L;
+  p.P = prefix_len;
+  p.B = B;
+  p.nPblk = pl.nPblk;
+  p.nKblk = pl.nKblk;
+  p.num_pages = num_pages;
+  p.n_splits = pl.n_splits;
+  p.nqs = pl.nqs;
+  p.out_f32 = dtype == CA_DTYPE_FP32 ? 1 : 0;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  p.wait_ns = kWaitNs;
+  const int grid = Hkv * pl.nhalves * pl.nqs * pl.n_splits;
+  e = launch_chunk_attention(tq, tqlo, tk, tv, p, D, pl.NT, dtype == CA_DTYPE_FP32, grid, st);
+  if (e != cudaSuccess) return cuda_fail(e, "ca_chunk_attention launch");
+  if (pl.n_splits > 1) {
+    e = launch_split_combine(p.Opart, p.LSEpart, pl.n_splits, L, Hq, D, O, LSE, p.out_f32, st);
+    if (e != cudaSuccess) return cuda_fail(e, "ca_chunk_attention combine launch");
+  }
+  return CA_OK;
+}
+
+int ca_check(int32_t* err_flag, void* stream) {
+  if (!err_flag) return fail(CA_ERR_ARG, "ca_check: null err_flag");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, err_flag, sizeof(h), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(err_flag, 0, sizeof(int32_t), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "ca_check");
+  if (h & CA_FLAG_TIMEOUT) return fail(CA_ERR_TIMEOUT, "device: a pipeline wait timed out");
+  if (h & CA_FLAG_BOUNDS)
+    return fail(CA_ERR_BOUNDS, "device: table entry, count or page id out of range");
+  return CA_OK;
+}
+
+int ca_wait_probe(int32_t* err_flag, int limit_us, void* stream) {
+  if (!err_flag || limit_us < 1 || limit_us > 10000000)
+    return fail(CA_ERR_ARG, "ca_wait_probe: need err_flag and 1 <= limit_us <= 1e7");
+  cudaError_t e =
+      launch_wait_probe(err_flag, (unsigned long long)limit_us * 1000ull, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "ca_wait_probe launch");
+  return CA_OK;
+}
+
+}  // extern "C"

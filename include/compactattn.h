@@ -1,0 +1,153 @@
+/*
+ * compactattn.h — C ABI of libcompactattn.so: Block-Union KV selection and
+ * chunked-prefill attention over the selected blocks of a paged KV cache, for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Method: "CompactAttention: Accelerating Chunked Prefill with Block-Union KV
+ * Selection", Abstract.  Per chunk, a 2D block-sparse mask of every query head
+ * is used as a KV-selection signal: the mask is OR-ed over the chunk's
+ * Q-blocks (Q-block union) and over the query heads that share one KV head
+ * (intra-group union), giving one minimal, sorted KV block table per KV head.
+ * The chunk's queries then attend to exactly the KV blocks of their group's
+ * table, read in place from the paged cache (no KV compaction).
+ *
+ * Conventions for every call:
+ *   - returns CA_OK (0) or a negative CA_ERR_* code; ca_last_error() gives text;
+ *   - every pointer argument is a DEVICE pointer owned by the caller, except
+ *     where a call says otherwise; the library allocates no device memory;
+ *   - every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream); argument errors are reported before anything is
+ *     launched, device-side errors through `err_flag`;
+ *   - all arrays are C-contiguous with the shapes given below;
+ *   - thread safety: calls may come from several host threads; the tensor-map
+ *     encoder entry point is resolved once under a lock.
+ *
+ * Notation: Hq query heads, Hkv KV heads, G = Hq / Hkv heads per group; query
+ * head h belongs to group h / G.  B = block = page size in tokens.
+ * P = prefix_len, L = chunk_len, nQblk = L / B, nKblk = (P + L) / B.
+ */
+#ifndef COMPACTATTN_H
+#define COMPACTATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CA_OK 0
+#define CA_ERR_ARG (-1)       /* bad shape, size or null pointer             */
+#define CA_ERR_ALIGN (-2)     /* prefix/chunk not a multiple of the block    */
+#define CA_ERR_DTYPE (-3)     /* unsupported dtype code                       */
+#define CA_ERR_LAUNCH (-4)    /* a CUDA launch or runtime call failed        */
+#define CA_ERR_BOUNDS (-5)    /* device: table entry or page id out of range */
+#define CA_ERR_TIMEOUT (-6)   /* device: a bounded pipeline wait ran out     */
+#define CA_ERR_WORKSPACE (-7) /* workspace missing or too small              */
+
+/* Bits a kernel ORs into *err_flag (device int32). */
+#define CA_FLAG_BOUNDS 1
+#define CA_FLAG_TIMEOUT 2
+
+#define CA_DTYPE_BF16 0
+#define CA_DTYPE_FP32 1
+
+/*
+ * ca_build_tables — Q-block union + intra-group union + compaction
+ * ("CompactAttention ...", Abstract: masks become GQA-aware per-group KV
+ * block tables, the minimal ones that keep every selected KV block).
+ *
+ *   mask    uint8 [Hq, nQblk, nKblk]; nonzero = KV block kb selected for
+ *           (head h, Q-block qb).  Read as-is: bits above the causal diagonal
+ *           are kept (attention's causal rule makes them inert).
+ *   tables  int32 [Hkv, nKblk] (out): row g holds the ascending ids of every
+ *           block selected by any (h in group g, qb), then -1 padding.
+ *   counts  int32 [Hkv] (out): number of valid entries of each row.
+ * Limits: 1 <= Hkv <= Hq, Hq % Hkv == 0, nQblk >= 1, 1 <= nKblk <= 65536.
+ * The result is bit-exact and deterministic.
+ */
+int ca_build_tables(const uint8_t* mask, int Hq, int Hkv, int nQblk, int nKblk,
+                    int32_t* tables, int32_t* counts, void* stream);
+
+/*
+ * ca_build_tables_batched — the same for nb independent masks in one launch
+ * (e.g. one mask per layer): masks [nb, Hq, nQblk, nKblk] -> tables
+ * [nb, Hkv, nKblk], counts [nb, Hkv].  1 <= nb <= 65535.
+ */
+int ca_build_tables_batched(const uint8_t* masks, int nb, int Hq, int Hkv, int nQblk,
+                            int nKblk, int32_t* tables, int32_t* counts, void* stream);
+
+/*
+ * ca_workspace_size — bytes of device workspace ca_chunk_attention needs for
+ * these shapes: bf16 copies of fp32 inputs (dtype == CA_DTYPE_FP32) and the
+ * fp32 partial results of a KV-range split (n_splits > 1; n_splits <= 0
+ * means the split ca_chunk_attention picks by itself).  Returns 0 when none
+ * is needed, and (size_t)-1 for invalid shapes.
+ */
+size_t ca_workspace_size(int dtype, int Hq, int Hkv, int head_dim, int block, int chunk_len,
+                         int prefix_len, int num_pages, int n_splits);
+
+/*
+ * ca_chunk_attention — attention of one prefill chunk over the blocks of its
+ * group tables, read in place from a paged KV cache ("CompactAttention ...",
+ * Abstract: selected KV blocks accessed in place without KV compaction).
+ *
+ * For query head h (group g = h / G) and chunk query i at position p = P + i:
+ *   keys    J = { j : j / B in tables[g][0 .. counts[g]),  j <= p }
+ *   LSE[h,i] = ln sum_{j in J} exp(s_j),  s_j = Q[i,h] . K(j) / sqrt(head_dim)
+ *   O[i,h]   = sum_{j in J} exp(s_j - LSE[h,i]) V(j)
+ * with K(j) = K_pages[page_table[j / B], g, j % B, :] (V alike).  An empty J
+ * gives O = 0 and LSE = -inf.
+ *
+ *   Q           [L, Hq, d], dtype `dtype` (bf16 or fp32).  The tensor cores
+ *               take bf16: an fp32 Q is carried as two bf16 terms
+ *               (hi = rn(Q), lo = rn(Q - hi)) so that its rounding does not
+ *               shift whole score rows; fp32 K and V are rounded to bf16
+ *               (round to nearest even), on the device, into the workspace
+ *   K_pages,
+ *   V_pages     [num_pages, Hkv, B, d], dtype `dtype`; the chunk's own keys
+ *               must already be in their pages
+ *   page_table  int32 [nKblk]: logical block -> physical page
+ *   tables,
+ *   counts      as written by ca_build_tables for this chunk (ascending rows)
+ *   O           [L, Hq, d] (out), dtype `dtype`
+ *   LSE         float32 [Hq, L] (out), natural log
+ *   workspace   >= ca_workspace_size(...) bytes (may be NULL if that is 0)
+ *   n_splits    KV-range splits per work unit (<= 0: automatic)
+ *   err_flag    int32 (device, may be NULL): the kernels OR CA_FLAG_* into it
+ *               on an out-of-range table entry / page id (the access is
+ *               clamped, results are then undefined) or on a pipeline wait
+ *               that exceeded its time limit.  Read it with ca_check().
+ * Limits: head_dim in {64, 128}; block in {64, 128}; P % B == 0, L % B == 0,
+ * L >= 64; Hq % Hkv == 0; num_pages >= nKblk.
+ */
+int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, int dtype,
+                       int num_pages, const int32_t* page_table, const int32_t* tables,
+                       const int32_t* counts, int Hq, int Hkv, int head_dim, int block,
+                       int chunk_len, int prefix_len, void* O, float* LSE, void* workspace,
+                       size_t ws_bytes, int n_splits, int32_t* err_flag, void* stream);
+
+/*
+ * ca_check — synchronise `stream`, read *err_flag (device int32), clear it,
+ * and map it to CA_OK / CA_ERR_BOUNDS / CA_ERR_TIMEOUT.
+ */
+int ca_check(int32_t* err_flag, void* stream);
+
+/*
+ * ca_wait_probe — launch one CTA that waits on a pipeline barrier nobody
+ * signals, with a time limit of limit_us microseconds; on expiry it ORs
+ * CA_FLAG_TIMEOUT into *err_flag and returns.  Exercises the timeout path of
+ * every bounded wait without faulting or hanging the device.
+ */
+int ca_wait_probe(int32_t* err_flag, int limit_us, void* stream);
+
+/* Copy the last error message of the calling thread into buf (NUL-terminated). */
+int ca_last_error(char* buf, size_t n);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int ca_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* COMPACTATTN_H */

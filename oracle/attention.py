@@ -30,6 +30,14 @@ def depage(pages, page_table, nKblk):
     return out
 
 
+def _page(pages, p, g):
+    """One [B, d] page as float64; accepts numpy arrays or torch CPU tensors (e.g. bf16)."""
+    x = pages[p, g]
+    if hasattr(x, "double"):
+        return x.double().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
 def _key_ids(table_row, count, B):
     blocks = np.asarray(table_row[:count], dtype=np.int64)
     return (blocks[:, None] * B + np.arange(B)[None, :]).reshape(-1)
@@ -84,8 +92,8 @@ def oracle_chunk_attention(Q, K_pages, V_pages, page_table, tables, counts, pref
 def oracle_rows(Q, K_pages, V_pages, page_table, tables, counts, prefix_len, rows):
     """The same definition for a sample of (h, i) rows only.
 
-    Reads just the pages of the group's selected blocks, so it stays cheap at
-    full 128K size.  Returns O [len(rows), d] and LSE [len(rows)].
+    Reads just the pages of one group's selected blocks at a time, so it stays
+    cheap at full 128K size.  Returns O [len(rows), d] and LSE [len(rows)].
     """
     Q = np.asarray(Q)
     L_c, Hq, d = Q.shape
@@ -93,23 +101,24 @@ def oracle_rows(Q, K_pages, V_pages, page_table, tables, counts, prefix_len, row
     G = Hq // Hkv
     O = np.zeros((len(rows), d))
     LSE = np.full(len(rows), -np.inf)
-    cache = {}
+    by_group = {}
     for r, (h, i) in enumerate(rows):
-        g = h // G
-        if g not in cache:
-            cnt = int(counts[g])
-            blocks = np.asarray(tables[g][:cnt], dtype=np.int64)
-            Kg = np.concatenate([np.asarray(K_pages[int(page_table[kb]), g], dtype=np.float64)
-                                 for kb in blocks], axis=0) if cnt else np.zeros((0, d))
-            Vg = np.concatenate([np.asarray(V_pages[int(page_table[kb]), g], dtype=np.float64)
-                                 for kb in blocks], axis=0) if cnt else np.zeros((0, d))
-            J = _key_ids(tables[g], cnt, B)
-            cache[g] = (Kg, Vg, J)
-        Kg, Vg, J = cache[g]
-        q = np.asarray(Q[i, h], dtype=np.float64)[None]
-        o, lse = _attend(q, Kg, Vg, J, np.array([prefix_len + i]), d)
-        O[r] = o[0]
-        LSE[r] = lse[0]
+        by_group.setdefault(h // G, []).append(r)
+    for g, idx in by_group.items():
+        cnt = int(counts[g])
+        blocks = np.asarray(tables[g][:cnt], dtype=np.int64)
+        if cnt:
+            Kg = np.concatenate([_page(K_pages, int(page_table[kb]), g) for kb in blocks], axis=0)
+            Vg = np.concatenate([_page(V_pages, int(page_table[kb]), g) for kb in blocks], axis=0)
+        else:
+            Kg = Vg = np.zeros((0, d))
+        J = _key_ids(tables[g], cnt, B)
+        for r in idx:
+            h, i = rows[r]
+            q = np.asarray(Q[i, h], dtype=np.float64)[None]
+            o, lse = _attend(q, Kg, Vg, J, np.array([prefix_len + i]), d)
+            O[r] = o[0]
+            LSE[r] = lse[0]
     return O, LSE
 
 

@@ -1,0 +1,105 @@
+"""Host-side tests of the C ABI (no GPU): the library builds, loads, exports
+every symbol include/compactattn.h declares, and rejects bad arguments before
+launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bsc():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_bsc_build", os.path.join(ROOT, "block_sparse_chunked_b200", "_build.py"))
+    m = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(m)
+    m.build_library()
+    import block_sparse_chunked_b200
+    return block_sparse_chunked_b200
+
+
+def header_symbols():
+    src = open(os.path.join(ROOT, "include", "compactattn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|size_t)\s+(ca_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_expected_calls():
+    syms = header_symbols()
+    for s in ["ca_build_tables", "ca_build_tables_batched", "ca_workspace_size",
+              "ca_chunk_attention", "ca_check", "ca_last_error"]:
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(bsc):
+    lib = ctypes.CDLL(bsc.LIB_PATH)
+    for s in header_symbols():
+        assert hasattr(lib, s), s
+    assert set(header_symbols()) <= set(bsc.EXPORTS)
+
+
+def test_version(bsc):
+    assert bsc.version() == 100
+
+
+FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("Hq,Hkv,nQ,nK,nb", [(6, 4, 2, 10, 1), (4, 0, 2, 10, 1), (4, 2, 0, 10, 1),
+                                              (4, 2, 2, 0, 1), (4, 2, 2, 65537, 1),
+                                              (4, 2, 2, 10, 0), (4, 8, 2, 10, 1)])
+def test_build_tables_rejects_bad_shapes(bsc, Hq, Hkv, nQ, nK, nb):
+    rc = bsc.lib.ca_build_tables_batched(FAKE, nb, Hq, Hkv, nQ, nK, FAKE, FAKE, None)
+    assert rc == bsc.CA_ERR_ARG
+    assert "ca_build_tables" in bsc.last_error()
+
+
+def test_build_tables_rejects_null(bsc):
+    assert bsc.lib.ca_build_tables(None, 4, 2, 2, 10, FAKE, FAKE, None) == bsc.CA_ERR_ARG
+
+
+def _attn(bsc, **kw):
+    a = dict(Q=FAKE, K=FAKE, V=FAKE, dtype=0, num_pages=20, pt=FAKE, tables=FAKE, counts=FAKE,
+             Hq=4, Hkv=1, d=64, B=64, L=256, P=1024, O=FAKE, LSE=FAKE, ws=None, wsn=0, S=1,
+             err=None)
+    a.update(kw)
+    return bsc.lib.ca_chunk_attention(a["Q"], a["K"], a["V"], a["dtype"], a["num_pages"], a["pt"],
+                                      a["tables"], a["counts"], a["Hq"], a["Hkv"], a["d"], a["B"],
+                                      a["L"], a["P"], a["O"], a["LSE"], a["ws"], a["wsn"], a["S"],
+                                      a["err"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Q=None), -1), (dict(dtype=7), -3), (dict(P=1000), -2), (dict(L=100), -2),
+    (dict(B=32), -1), (dict(d=96), -1), (dict(Hq=6, Hkv=4), -1), (dict(num_pages=19), -1),
+    (dict(Q=ctypes.c_void_p(0x1001)), -1), (dict(dtype=1), -7), (dict(S=4), -7),
+])
+def test_chunk_attention_rejects_bad_arguments(bsc, kw, code):
+    assert _attn(bsc, **kw) == code
+    assert bsc.last_error()
+
+
+def test_workspace_size_rules(bsc):
+    ws = bsc.lib.ca_workspace_size
+    # bf16, >= one CTA per SM of units: no split, no workspace
+    assert ws(0, 32, 8, 128, 64, 2048, 129024, 2048, 0) == 0
+    # explicit split: fp32 partials + LSE partials
+    n = ws(0, 32, 8, 128, 64, 2048, 129024, 2048, 2)
+    assert n >= 2 * 2048 * 32 * 128 * 4 + 2 * 32 * 2048 * 4
+    # fp32 input adds bf16 copies of Q, K and V
+    assert ws(1, 4, 1, 64, 64, 256, 1024, 20, 1) >= (256 * 4 * 64 + 2 * 20 * 64 * 64) * 2
+    assert ws(0, 4, 3, 64, 64, 256, 1024, 20, 1) == ctypes.c_size_t(-1).value
+
+
+def test_check_and_probe_reject_null(bsc):
+    assert bsc.lib.ca_check(None, None) == bsc.CA_ERR_ARG
+    assert bsc.lib.ca_wait_probe(None, 10, None) == bsc.CA_ERR_ARG
+
+
+def test_accounting_dense_128k(bsc):
+    # 32 heads x sum_{qb<32} (2016 + qb + 1) pairs x 4 * 64^2 * 128 FLOPs
+    assert bsc.dense_flops(32, 2016, 32, 64, 128) == 4 * 64 * 64 * 128 * 32 * (32 * 2017 + 496)
