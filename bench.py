@@ -204,11 +204,14 @@ def reference_arm(args, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sets", type=int, default=4)
+    ap.add_argument("--skip-extras", action="store_true",
+                    help="time the step only (no dense path, batched builder, e2e): the small "
+                         "case used for ncu captures")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -293,6 +296,15 @@ def main():
     mean_step, mean_attn = float(tot[0]), float(tot[1])
     value = world * mean_flops / (mean_step * 1e-3) / 1e12
     attn_tflops = mean_flops / (mean_attn * 1e-3) / 1e12
+
+    if args.skip_extras:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": world * mean_flops / (mean_step * 1e-3) / 1e12,
+                              "unit": "TFLOP/s", "ms_per_step": mean_step, "attention_ms": mean_attn,
+                              "note": "step only (--skip-extras)"}), flush=True)
+        if pg:
+            pg.destroy_process_group()
+        return
 
     # ---- density-100% path on the same shapes (all blocks selected)
     dense_t = torch.arange(w.nKblk, dtype=torch.int32, device=dev).repeat(w.Hkv, 1).contiguous()
