@@ -209,6 +209,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sets", type=int, default=4)
+    ap.add_argument("--builder-only", type=int, default=0, metavar="NB",
+                    help="only run the batched table builder on NB 128K masks per launch "
+                         "(the case used for the builder's ncu capture) and exit")
     ap.add_argument("--skip-extras", action="store_true",
                     help="time the step only (no dense path, batched builder, e2e): the small "
                          "case used for ncu captures")
@@ -244,6 +247,28 @@ def main():
 
     peaks, peak_src = load_peaks()
     w = workloads.get_config("ctx128k")
+    if args.builder_only:
+        nb = args.builder_only
+        base = workloads.mask_for(w, seed=0)
+        rng = np.random.default_rng(1)
+        # distinct masks: each one a random column rotation of the seeded mask
+        masks = torch.from_numpy(np.stack([np.roll(base, int(r), axis=2)
+                                           for r in rng.integers(0, w.nKblk, nb)])).to(dev)
+        tb = torch.empty(nb, w.Hkv, w.nKblk, dtype=torch.int32, device=dev)
+        cb = torch.empty(nb, w.Hkv, dtype=torch.int32, device=dev)
+        ts = []
+        for i in range(args.warmup + args.steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            bsc.build_tables_batched(masks, w.Hkv, tb, cb)
+            b.record()
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                ts.append(a.elapsed_time(b))
+        nbytes = bsc.builder_bytes(nb, w.Hq, w.Hkv, w.nQblk, w.nKblk)
+        print(json.dumps({"builder_masks": nb, "bytes": nbytes, "us": statistics.mean(ts) * 1e3,
+                          "GB/s": nbytes / (statistics.mean(ts) * 1e-3) / 1e9}), flush=True)
+        return
     x, sets = make_sets(w, args.sets, dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     ws_n = bsc.workspace_size(torch.bfloat16, w.Hq, w.Hkv, w.head_dim, w.block, w.chunk_len,
