@@ -29,6 +29,10 @@ EXPORTS = {
     "ca_chunk_attention": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _vp, _c_int, _c_int,
                                     _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_size,
                                     _c_int, _vp, _vp]),
+    "ca_chunk_attention_noalloc": (_c_int, [_vp, _vp, _vp, _c_int, _vp, _vp, _vp, _c_int, _c_int,
+                                            _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int,
+                                            _vp, _vp]),
+    "ca_noalloc_scratch_bytes": (_c_size, []),
     "ca_check": (_c_int, [_vp, _vp]),
     "ca_wait_probe": (_c_int, [_vp, _c_int, _vp]),
     "ca_last_error": (_c_int, [ctypes.c_char_p, _c_size]),

@@ -122,6 +122,9 @@ WsLayout ws_layout(int dtype, int Hq, int Hkv, int D, int B, int L, int num_page
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
+
+void set_last_error(const char* msg) { g_last_error = msg ? msg : ""; }
+
 }  // namespace ca
 
 using namespace ca;

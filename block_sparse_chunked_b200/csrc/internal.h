@@ -37,4 +37,7 @@ cudaError_t launch_split_f32_bf16(const float* src, void* hi, void* lo, size_t n
                                   cudaStream_t st);
 cudaError_t launch_wait_probe(int32_t* err, unsigned long long limit_ns, cudaStream_t st);
 
+// Record a message for ca_last_error() on the calling thread.
+void set_last_error(const char* msg);
+
 }  // namespace ca

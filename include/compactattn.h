@@ -128,6 +128,42 @@ int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, 
                        size_t ws_bytes, int n_splits, int32_t* err_flag, void* stream);
 
 /*
+ * ca_chunk_attention_noalloc — ca_chunk_attention (bf16 inputs) for callers
+ * that cannot allocate device memory.  The paper has no counterpart: this is
+ * a deployment variant of the same computation.
+ *
+ * Who needs it: code that runs under an allocator it does not own (e.g. an
+ * inference engine that reserves the whole GPU at start-up and forbids
+ * cudaMalloc in its forward pass) or a latency-critical loop in which an
+ * allocation, and the synchronisation it can imply, is not allowed.  With
+ * n_splits > 1 the regular entry point needs caller workspace for the split
+ * partials; here they go to a scratch array compiled into the library
+ * (ca_noalloc_scratch_bytes() bytes, 32 MiB, which every GPU that loads the
+ * library keeps allocated until the process exits).  The caller passes only
+ * inputs and outputs; arguments mean what they mean for ca_chunk_attention,
+ * with dtype fixed to CA_DTYPE_BF16.
+ *
+ *   - Shapes whose split partials exceed the scratch size are rejected with
+ *     CA_ERR_WORKSPACE (nothing is launched); n_splits <= 0 picks the split
+ *     as ca_chunk_attention does.
+ *   - The first call on each device looks up the scratch array's device
+ *     address (cudaGetSymbolAddress, with that device current); make that
+ *     first call before any stream capture.
+ *   - All calls on a device share the scratch and it keeps the last call's
+ *     contents (nothing in it needs to start at zero).  Calls whose kernels
+ *     overlap on the GPU race on it: do not run two at once on one device.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ */
+int ca_chunk_attention_noalloc(const void* Q, const void* K_pages, const void* V_pages,
+                               int num_pages, const int32_t* page_table, const int32_t* tables,
+                               const int32_t* counts, int Hq, int Hkv, int head_dim, int block,
+                               int chunk_len, int prefix_len, void* O, float* LSE, int n_splits,
+                               int32_t* err_flag, void* stream);
+
+/* Size in bytes of the fixed scratch array ca_chunk_attention_noalloc uses. */
+size_t ca_noalloc_scratch_bytes(void);
+
+/*
  * ca_check — synchronise `stream`, read *err_flag (device int32), clear it,
  * and map it to CA_OK / CA_ERR_BOUNDS / CA_ERR_TIMEOUT.
  */
