@@ -339,7 +339,7 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
     const uint32_t tS = tmem + lane_off + 256 + t * 128;
     const uint32_t tO = tmem + lane_off + t * 128;
     const int diag_lim = (t0 % p.B) + (row & 63);  // visible keys of the diagonal block: jl <= this
-    float m_used = -INFINITY, l = 0.f;
+    float m_used = -INFINITY, l0 = 0.f, l1 = 0.f;
     bool ok = true;
     for (int j = 0; j < nloc; ++j) {
       const int stage = s0 + j;
@@ -350,32 +350,59 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
       ok = wait_warp(s_full(t), j & 1, p, abort_flag);
       if (!ok) break;
       tc_fence_after();
-      // pass 1: row max of the scaled, masked scores (32 columns at a time)
-      float mx = -INFINITY;
-      uint32_t r[32];
+      // One TMEM pass: the row's scores (raw Q.K) into registers.
+      float sr[kStageKeys];
+      tmem_ld64f(tS, sr);
+      if (nvalid > 64) tmem_ld64f(tS + 64, sr + 64);
+      tmem_wait_ld();
+      if (nvalid <= 64) {
 #pragma unroll
-      for (int c = 0; c < kStageKeys / 32; ++c) {
-        if (c * 32 < nvalid) {
-          tmem_ld32(tS + c * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int col = c * 32 + i;
-            float x = __uint_as_float(r[i]) * p.scale_log2;
-            if (diag_stage && col >= diag_c0 && (col - diag_c0) > diag_lim) x = -INFINITY;
-            mx = fmaxf(mx, x);
-          }
-        }
+        for (int c = 64; c < kStageKeys; ++c) sr[c] = -INFINITY;
       }
+      if (diag_stage) {  // token-level causal mask, diagonal block only
+#pragma unroll
+        for (int c = 0; c < kStageKeys; ++c)
+          if (c >= diag_c0 && (c - diag_c0) > diag_lim) sr[c] = -INFINITY;
+      }
+      // row max of the raw scores (scale > 0 commutes with max)
+      float mx0 = max3(sr[0], sr[1], sr[2]);
+      float mx1 = max3(sr[3], sr[4], sr[5]);
+#pragma unroll
+      for (int c = 6; c < kStageKeys - 2; c += 4) {
+        mx0 = max3(mx0, sr[c], sr[c + 1]);
+        mx1 = max3(mx1, sr[c + 2], sr[c + 3]);
+      }
+      const float mx = max3(mx0, mx1, fmaxf(sr[kStageKeys - 2], sr[kStageKeys - 1])) * p.scale_log2;
       const float m_new = fmaxf(m_used, mx);
       const bool need = (m_new != -INFINITY) && (m_new > m_used + 8.0f);
       float alpha = 1.f;
       if (need) {
         alpha = ex2(m_used - m_new);  // 0 when m_used == -inf
-        l *= alpha;
+        l0 *= alpha;
+        l1 *= alpha;
         m_used = m_new;
       }
+      const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
+      const float sc = p.scale_log2;
+      // p = 2^(s*scale - m): packed FMA, then ex2; fp32 row sum before the bf16 rounding
+#pragma unroll
+      for (int c = 0; c < kStageKeys / 32; ++c) {
+        if (c * 32 < nvalid) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float x0, x1;
+            ffma2(x0, x1, sr[c * 32 + 2 * i], sr[c * 32 + 2 * i + 1], sc, sc, nm, nm);
+            const float e0 = ex2(x0), e1 = ex2(x1);
+            fadd2(l0, l1, e0, e1);
+            pk[i] = pack_bf16x2(e0, e1);
+          }
+          tmem_st16(tS + c * 16, pk);
+        }
+      }
+      // O still holds the sum over earlier stages at the old max: bring it to the new one
       if (__any_sync(0xffffffffu, need) && j > 0) {
+        uint32_t r[32];
         for (int c = 0; c < D / 32; ++c) {
           tmem_ld32(tO + c * 32, r);
           tmem_wait_ld();
@@ -384,34 +411,12 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
           tmem_st32(tO + c * 32, r);
         }
       }
-      const float msub = (m_used == -INFINITY) ? 0.f : m_used;
-      // pass 2: p = 2^(x - m), row sum in fp32, P as bf16 pairs back over S
-#pragma unroll
-      for (int c = 0; c < kStageKeys / 32; ++c) {
-        if (c * 32 < nvalid) {
-          tmem_ld32(tS + c * 32, r);
-          tmem_wait_ld();
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int col = c * 32 + 2 * i;
-            float x0 = __uint_as_float(r[2 * i]) * p.scale_log2;
-            float x1 = __uint_as_float(r[2 * i + 1]) * p.scale_log2;
-            if (diag_stage && col >= diag_c0 && (col - diag_c0) > diag_lim) x0 = -INFINITY;
-            if (diag_stage && col + 1 >= diag_c0 && (col + 1 - diag_c0) > diag_lim) x1 = -INFINITY;
-            const float a = ex2(x0 - msub);
-            const float b = ex2(x1 - msub);
-            l += a + b;
-            pk[i] = pack_bf16x2(a, b);
-          }
-          tmem_st16(tS + c * 16, pk);
-        }
-      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full(t));
     }
     // ---- epilogue
+    const float l = l0 + l1;
     if (ok && nloc > 0) ok = wait_warp(o_done, 0, p, abort_flag);
     if (ok && nloc > 0) tc_fence_after();
     const bool have = ok && nloc > 0 && l > 0.f;
