@@ -46,6 +46,7 @@ namespace ca {
 constexpr int kStageKeys = 128;
 
 
+
 __device__ __forceinline__ void set_flag(int32_t* err, int f) {
   if (err) atomicOr(err, f);
 }
@@ -182,25 +183,33 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
 
   if (warp == 0) {
     // ================================================================ producer
-    if (lane == 0 && nloc > 0) {
-      prefetch_tmap(&tmQ);
-      if (QSPLIT) prefetch_tmap(&tmQlo);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
+    // The whole warp runs the loop: lane i prefetches table entry i of the next
+    // group of 32 and its page id, so the dependent lookups tables ->
+    // page_table are off the per-stage path; lane 0 issues the copies.
+    if (nloc > 0) {
       const uint64_t pol = policy_evict_last();
-      mbar_expect_tx(q_full, S::kQTerms * NT * 128 * D * 2);
-      for (int q = 0; q < S::kQTerms; ++q)
-        for (int t = 0; t < NT; ++t)
-          for (int s = 0; s < 2; ++s) {
-            int hl = hh * p.HPU + 2 * t + s;  // head within the group
-            const int hcap = min(p.G - 1, hh * p.HPU + p.HPU - 1);
-            hl = min(hl, hcap);
-            const int head = g * p.G + hl;
-            for (int c = 0; c < KCH; ++c)
-              tma_load_3d(sbase + S::kQOff + (q * NT + t) * S::kQTile + c * S::kChunkBytes +
-                              s * 64 * 128,
-                          q ? &tmQlo : &tmQ, q_full, c * 64, head, t0);
-          }
+      if (lane == 0) {
+        prefetch_tmap(&tmQ);
+        if (QSPLIT) prefetch_tmap(&tmQlo);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        mbar_expect_tx(q_full, S::kQTerms * NT * 128 * D * 2);
+        for (int q = 0; q < S::kQTerms; ++q)
+          for (int t = 0; t < NT; ++t)
+            for (int s = 0; s < 2; ++s) {
+              int hl = hh * p.HPU + 2 * t + s;  // head within the group
+              const int hcap = min(p.G - 1, hh * p.HPU + p.HPU - 1);
+              hl = min(hl, hcap);
+              const int head = g * p.G + hl;
+              for (int c = 0; c < KCH; ++c)
+                tma_load_3d(sbase + S::kQOff + (q * NT + t) * S::kQTile + c * S::kChunkBytes +
+                                s * 64 * 128,
+                            q ? &tmQlo : &tmQ, q_full, c * 64, head, t0);
+            }
+      }
+      const int e_begin = s0 * spb;
+      const int e_end = min(n_live, (s0 + nloc) * spb);
+      int pg_cache = 0, cache_base = -32;
       bool ok = true;
       for (int j = 0; j < nloc && ok; ++j) {
         const int stage = s0 + j, slot = j % kNS, round = j / kNS;
@@ -208,122 +217,141 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
         const uint32_t bytes = (uint32_t)npg * p.B * D * 2;
         int page[2] = {0, 0};
         for (int pi = 0; pi < npg; ++pi) {
-          int kb = trow[stage * spb + pi];
-          if (kb < 0 || kb >= p.nKblk) {
-            set_flag(p.err, CA_FLAG_BOUNDS);
-            kb = 0;
+          const int e = stage * spb + pi;
+          if (e >= cache_base + 32) {  // refill: 32 entries, one per lane
+            cache_base = e;
+            const int my = e + lane;
+            int pg = 0;
+            if (my < e_end && my >= e_begin) {
+              int kb = trow[my];
+              if (kb < 0 || kb >= p.nKblk) {
+                set_flag(p.err, CA_FLAG_BOUNDS);
+                kb = 0;
+              }
+              pg = p.page_table[kb];
+              if (pg < 0 || pg >= p.num_pages) {
+                set_flag(p.err, CA_FLAG_BOUNDS);
+                pg = 0;
+              }
+            }
+            pg_cache = pg;
           }
-          int pg = p.page_table[kb];
-          if (pg < 0 || pg >= p.num_pages) {
-            set_flag(p.err, CA_FLAG_BOUNDS);
-            pg = 0;
-          }
-          page[pi] = pg;
+          page[pi] = __shfl_sync(0xffffffffu, pg_cache, e - cache_base);
         }
-        if (round > 0) ok = (*abort_flag == 0) && mbar_wait(empty_k(slot), (round - 1) & 1, p.wait_ns);
-        if (!ok) break;
-        mbar_expect_tx(full_k(slot), bytes);
-        for (int pi = 0; pi < npg; ++pi)
-          for (int c = 0; c < KCH; ++c)
-            tma_load_4d(sbase + S::kKOff + slot * S::kKV + c * S::kChunkBytes + pi * p.B * 128,
-                        &tmK, full_k(slot), c * 64, 0, g, page[pi], pol);
-        if (round > 0) ok = (*abort_flag == 0) && mbar_wait(empty_v(slot), (round - 1) & 1, p.wait_ns);
-        if (!ok) break;
-        mbar_expect_tx(full_v(slot), bytes);
-        for (int pi = 0; pi < npg; ++pi)
-          for (int c = 0; c < KCH; ++c)
-            tma_load_4d(sbase + S::kVOff + slot * S::kKV + c * S::kChunkBytes + pi * p.B * 128,
-                        &tmV, full_v(slot), c * 64, 0, g, page[pi], pol);
+        if (round > 0) ok = wait_warp(empty_k(slot), (round - 1) & 1, p, abort_flag);
+        if (ok) {
+          mbar_expect_tx_w(full_k(slot), bytes);
+          for (int pi = 0; pi < npg; ++pi)
+            for (int c = 0; c < KCH; ++c)
+              tma_load_4d_w(sbase + S::kKOff + slot * S::kKV + c * S::kChunkBytes + pi * p.B * 128,
+                            &tmK, full_k(slot), c * 64, 0, g, page[pi], pol);
+        }
+        if (ok && round > 0) ok = wait_warp(empty_v(slot), (round - 1) & 1, p, abort_flag);
+        if (ok) {
+          mbar_expect_tx_w(full_v(slot), bytes);
+          for (int pi = 0; pi < npg; ++pi)
+            for (int c = 0; c < KCH; ++c)
+              tma_load_4d_w(sbase + S::kVOff + slot * S::kKV + c * S::kChunkBytes + pi * p.B * 128,
+                            &tmV, full_v(slot), c * 64, 0, g, page[pi], pol);
+        }
       }
-      if (!ok && *abort_flag == 0) {
-        *abort_flag = 1;
-        set_flag(p.err, CA_FLAG_TIMEOUT);
-      }
-      // Do not leave with copies in flight: the last stages' loads must land.
-      for (int j = max(0, nloc - kNS); j < nloc; ++j) {
-        mbar_wait(full_k(j % kNS), (j / kNS) & 1, p.wait_ns);
-        mbar_wait(full_v(j % kNS), (j / kNS) & 1, p.wait_ns);
+      if (lane == 0) {
+        // Do not leave with copies in flight: the last stages' loads must land.
+        for (int j = max(0, nloc - kNS); j < nloc; ++j) {
+          mbar_wait(full_k(j % kNS), (j / kNS) & 1, p.wait_ns);
+          mbar_wait(full_v(j % kNS), (j / kNS) & 1, p.wait_ns);
+        }
       }
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
-    if (lane == 0 && nloc > 0) {
-      const uint32_t idesc_pv = idesc_bf16(128, D, 1);
+    // The whole warp runs this loop (addresses stay warp-uniform); one elected
+    // lane issues each tcgen05.mma / commit.
+    if (nloc > 0) {
+      // Descriptors differ per MMA only in the start-address field (address >> 4
+      // in bits 0-13): build each operand's descriptor once and add the
+      // compile-time byte offset >> 4 per K-step.
+      constexpr uint32_t kIdescPV = idesc_bf16(128, D, 1);
+      constexpr uint32_t kIdescS128 = idesc_bf16(128, 128, 0);
+      constexpr uint32_t kIdescS64 = idesc_bf16(128, 64, 0);
+      uint64_t qdesc[NT];
+#pragma unroll
+      for (int t = 0; t < NT; ++t) qdesc[t] = smem_desc_sw128(sbase + S::kQOff + t * S::kQTile, 16, 1024);
+      const uint64_t kdesc0 = smem_desc_sw128(sbase + S::kKOff, 16, 1024);
+      const uint64_t vdesc0 = smem_desc_sw128(sbase + S::kVOff, S::kChunkBytes, 1024);
       auto npg_of = [&](int j) { return min(spb, n_live - (s0 + j) * spb); };
       auto issue_s = [&](int t, int j) {
-        const int slot = j % kNS;
-        const int n = npg_of(j) * p.B;
-        const uint32_t idesc = idesc_bf16(128, n, 0);
-        const uint32_t qa = sbase + S::kQOff + t * S::kQTile;
-        const uint32_t kbase = sbase + S::kKOff + slot * S::kKV;
+        const uint64_t kd = kdesc0 + (uint64_t)(((j % kNS) * S::kKV) >> 4);
+        const uint32_t idesc = npg_of(j) * p.B == 128 ? kIdescS128 : kIdescS64;
+        const uint32_t dt = tmem + 256 + t * 128;
 #pragma unroll
         for (int q = 0; q < S::kQTerms; ++q)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * S::kChunkBytes + (kk & 3) * 32;
-            mma_ss(tmem + 256 + t * 128,
-                   smem_desc_sw128(qa + q * NT * S::kQTile + off, 16, 1024),
-                   smem_desc_sw128(kbase + off, 16, 1024), idesc, (q > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t off = ((kk >> 2) * S::kChunkBytes + (kk & 3) * 32) >> 4;
+            mma_ss_w(dt, qdesc[t] + (uint64_t)(((q * NT * S::kQTile) >> 4) + off), kd + off, idesc,
+                     (q > 0 || kk > 0) ? 1u : 0u);
           }
       };
       auto issue_pv = [&](int t, int j) {
-        const int slot = j % kNS;
-        const int ksteps = npg_of(j) * p.B / 16;
-        const uint32_t vbase = sbase + S::kVOff + slot * S::kKV;
-        for (int kk = 0; kk < ksteps; ++kk)
-          mma_ts(tmem + t * 128, tmem + 256 + t * 128 + kk * 8,
-                 smem_desc_sw128(vbase + kk * 16 * 128, S::kChunkBytes, 1024), idesc_pv,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+        const uint64_t vd = vdesc0 + (uint64_t)(((j % kNS) * S::kKV) >> 4);
+        const uint32_t dt = tmem + t * 128;
+        const uint32_t at = tmem + 256 + t * 128;
+        const uint32_t acc0 = j > 0 ? 1u : 0u;
+        if (npg_of(j) * p.B == 128) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts_w(dt, at + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), kIdescPV, kk > 0 ? 1u : acc0);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts_w(dt, at + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), kIdescPV, kk > 0 ? 1u : acc0);
+        }
       };
-      bool ok = (*abort_flag == 0) && mbar_wait(q_full, 0, p.wait_ns);
-      ok = ok && mbar_wait(full_k(0), 0, p.wait_ns);
+      bool ok = wait_warp(q_full, 0, p, abort_flag) && wait_warp(full_k(0), 0, p, abort_flag);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
-        mma_commit(s_full(0));
+        mma_commit_w(s_full(0));
         if (NT == 2) {
           issue_s(1, 0);
-          mma_commit(s_full(1));
+          mma_commit_w(s_full(1));
         }
-        mma_commit(empty_k(0));
+        mma_commit_w(empty_k(0));
       }
       for (int j = 0; j < nloc && ok; ++j) {
         const int slot = j % kNS;
-        ok = (*abort_flag == 0) && mbar_wait(p_full(0), j & 1, p.wait_ns) &&
-             mbar_wait(full_v(slot), (j / kNS) & 1, p.wait_ns);
+        ok = wait_warp(p_full(0), j & 1, p, abort_flag) &&
+             wait_warp(full_v(slot), (j / kNS) & 1, p, abort_flag);
         if (!ok) break;
         tc_fence_after();
         issue_pv(0, j);
         const bool more = j + 1 < nloc;
         if (more) {
-          ok = mbar_wait(full_k((j + 1) % kNS), ((j + 1) / kNS) & 1, p.wait_ns);
+          ok = wait_warp(full_k((j + 1) % kNS), ((j + 1) / kNS) & 1, p, abort_flag);
           if (!ok) break;
           tc_fence_after();
           issue_s(0, j + 1);
-          mma_commit(s_full(0));
+          mma_commit_w(s_full(0));
         }
         if (NT == 2) {
-          ok = (*abort_flag == 0) && mbar_wait(p_full(1), j & 1, p.wait_ns);
+          ok = wait_warp(p_full(1), j & 1, p, abort_flag);
           if (!ok) break;
           tc_fence_after();
           issue_pv(1, j);
         }
-        mma_commit(empty_v(slot));
+        mma_commit_w(empty_v(slot));
         if (more) {
           if (NT == 2) {
             issue_s(1, j + 1);
-            mma_commit(s_full(1));
+            mma_commit_w(s_full(1));
           }
-          mma_commit(empty_k((j + 1) % kNS));
+          mma_commit_w(empty_k((j + 1) % kNS));
         }
       }
-      if (!ok && *abort_flag == 0) {
-        *abort_flag = 1;
-        set_flag(p.err, CA_FLAG_TIMEOUT);
-      }
-      if (ok) mma_commit(o_done);
-      // every MMA issued by this thread has finished before TMEM is released
-      mma_commit(drain);
+      if (ok) mma_commit_w(o_done);
+      // every MMA issued by this warp has finished before TMEM is released
+      mma_commit_w(drain);
       mbar_wait(drain, 0, p.wait_ns);
     }
   } else if (warp >= 4) {
@@ -339,7 +367,7 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
     const uint32_t tS = tmem + lane_off + 256 + t * 128;
     const uint32_t tO = tmem + lane_off + t * 128;
     const int diag_lim = (t0 % p.B) + (row & 63);  // visible keys of the diagonal block: jl <= this
-    float m_used = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float m_used = -INFINITY, l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
     bool ok = true;
     for (int j = 0; j < nloc; ++j) {
       const int stage = s0 + j;
@@ -380,6 +408,8 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
         alpha = ex2(m_used - m_new);  // 0 when m_used == -inf
         l0 *= alpha;
         l1 *= alpha;
+        l2 *= alpha;
+        l3 *= alpha;
         m_used = m_new;
       }
       const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
@@ -394,7 +424,8 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
             float x0, x1;
             ffma2(x0, x1, sr[c * 32 + 2 * i], sr[c * 32 + 2 * i + 1], sc, sc, nm, nm);
             const float e0 = ex2(x0), e1 = ex2(x1);
-            fadd2(l0, l1, e0, e1);
+            if (i & 1) fadd2(l2, l3, e0, e1);  // two independent sum chains
+            else fadd2(l0, l1, e0, e1);
             pk[i] = pack_bf16x2(e0, e1);
           }
           tmem_st16(tS + c * 16, pk);
@@ -416,7 +447,7 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
       mbar_arrive(p_full(t));
     }
     // ---- epilogue
-    const float l = l0 + l1;
+    const float l = (l0 + l1) + (l2 + l3);
     if (ok && nloc > 0) ok = wait_warp(o_done, 0, p, abort_flag);
     if (ok && nloc > 0) tc_fence_after();
     const bool have = ok && nloc > 0 && l > 0.f;
