@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(s_full(t), 1);
-      mbar_init(p_full(t), 128);
+      mbar_init(p_full(t), 4);  // one arrival per softmax warp
     }
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
@@ -444,7 +444,8 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full(t));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full(t));
     }
     // ---- epilogue
     const float l = (l0 + l1) + (l2 + l3);
