@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -58,8 +59,11 @@ constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per pipeline wait
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+constexpr int kMaxPersistentUnits = 2048;  // units whose schedule a CTA keeps in shared memory
+
 struct Plan {
   int G, HPU, NT, nhalves, nqs, nPblk, nKblk, spb, n_splits;
+  int units, persistent, sk_ctas;
 };
 
 bool plan(int Hq, int Hkv, int head_dim, int block, int chunk_len, int prefix_len, int n_splits,
@@ -79,6 +83,21 @@ bool plan(int Hq, int Hkv, int head_dim, int block, int chunk_len, int prefix_le
   pl.spb = 128 / block;
   const long long units = (long long)Hkv * pl.nhalves * pl.nqs;
   const int max_stages = (pl.nKblk + pl.spb - 1) / pl.spb;
+  pl.units = (int)std::min<long long>(units, 0x7fffffff);
+  // Automatic mode: one CTA per unit when the units fill the SMs; otherwise a
+  // persistent grid of at most one CTA per SM, each taking an equal share of
+  // all units' KV stages (at least ~4 stages per CTA).  (At 256 units on 148
+  // SMs the persistent grid measured 5% slower than one CTA per unit: the
+  // piece boundaries and the merge cost more than the balance gains.)
+  pl.persistent = (n_splits <= 0 && units < kSMs && units <= kMaxPersistentUnits) ? 1 : 0;
+  if (n_splits <= 0 && !pl.persistent) n_splits = 1;
+  pl.sk_ctas = 0;
+  if (pl.persistent) {
+    const long long stages = units * max_stages;
+    pl.sk_ctas = (int)std::max<long long>(1, std::min<long long>(kSMs, stages / 4));
+    pl.n_splits = 1;
+    return true;
+  }
   int S = n_splits;
   if (S <= 0) {
     S = 1;
@@ -93,12 +112,23 @@ bool plan(int Hq, int Hkv, int head_dim, int block, int chunk_len, int prefix_le
 }
 
 struct WsLayout {
-  size_t opart = 0, lsepart = 0, q = 0, qlo = 0, k = 0, v = 0, total = 0;
+  size_t opart = 0, lsepart = 0, q = 0, qlo = 0, k = 0, v = 0, sched = 0, osk = 0, lsesk = 0,
+         total = 0;
 };
 
-WsLayout ws_layout(int dtype, int Hq, int Hkv, int D, int B, int L, int num_pages, int S) {
+WsLayout ws_layout(int dtype, int Hq, int Hkv, int D, int B, int L, int num_pages, const Plan& pl) {
   WsLayout w;
   size_t off = 0;
+  const int S = pl.n_splits;
+  if (pl.persistent) {
+    const size_t rows = (size_t)pl.NT * 128;
+    w.sched = off;
+    off = align256(off + (size_t)(pl.units + 1) * 4);
+    w.osk = off;
+    off = align256(off + 2 * (size_t)pl.sk_ctas * rows * D * 4);
+    w.lsesk = off;
+    off = align256(off + 2 * (size_t)pl.sk_ctas * rows * 4);
+  }
   if (S > 1) {
     w.opart = off;
     off = align256(off + (size_t)S * L * Hq * D * 4);
@@ -168,7 +198,7 @@ size_t ca_workspace_size(int dtype, int Hq, int Hkv, int head_dim, int block, in
   if (dtype != CA_DTYPE_BF16 && dtype != CA_DTYPE_FP32) return (size_t)-1;
   if (!plan(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl)) return (size_t)-1;
   if (num_pages < pl.nKblk) return (size_t)-1;
-  return ws_layout(dtype, Hq, Hkv, head_dim, block, chunk_len, num_pages, pl.n_splits).total;
+  return ws_layout(dtype, Hq, Hkv, head_dim, block, chunk_len, num_pages, pl).total;
 }
 
 int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, int dtype,
@@ -196,8 +226,7 @@ int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, 
     return fail(CA_ERR_ARG, "ca_chunk_attention: num_pages=%d < nKblk=%d", num_pages, pl.nKblk);
   if (!aligned16(Q) || !aligned16(K_pages) || !aligned16(V_pages) || !aligned16(O))
     return fail(CA_ERR_ARG, "ca_chunk_attention: Q, K_pages, V_pages and O must be 16-byte aligned");
-  const WsLayout wl =
-      ws_layout(dtype, Hq, Hkv, head_dim, block, chunk_len, num_pages, pl.n_splits);
+  const WsLayout wl = ws_layout(dtype, Hq, Hkv, head_dim, block, chunk_len, num_pages, pl);
   if (wl.total > 0 && (!workspace || ws_bytes < wl.total || !aligned16(workspace)))
     return fail(CA_ERR_WORKSPACE, "ca_chunk_attention: workspace of %zu bytes needed, got %zu",
                 wl.total, workspace ? ws_bytes : (size_t)0);
@@ -267,6 +296,12 @@ int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, 
   p.Opart = pl.n_splits > 1 ? reinterpret_cast<float*>(ws + wl.opart) : nullptr;
   p.LSEpart = pl.n_splits > 1 ? reinterpret_cast<float*>(ws + wl.lsepart) : nullptr;
   p.err = err_flag;
+  p.persistent = pl.persistent;
+  p.n_units = pl.units;
+  p.sk_ctas = pl.sk_ctas;
+  p.sk_sched = pl.persistent ? reinterpret_cast<int32_t*>(ws + wl.sched) : nullptr;
+  p.Osk = pl.persistent ? reinterpret_cast<float*>(ws + wl.osk) : nullptr;
+  p.LSEsk = pl.persistent ? reinterpret_cast<float*>(ws + wl.lsesk) : nullptr;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.G = pl.G;
@@ -283,9 +318,13 @@ int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, 
   p.out_f32 = dtype == CA_DTYPE_FP32 ? 1 : 0;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   p.wait_ns = kWaitNs;
-  const int grid = Hkv * pl.nhalves * pl.nqs * pl.n_splits;
+  const int grid = pl.persistent ? pl.sk_ctas : Hkv * pl.nhalves * pl.nqs * pl.n_splits;
   e = launch_chunk_attention(tq, tqlo, tk, tv, p, D, pl.NT, dtype == CA_DTYPE_FP32, grid, st);
   if (e != cudaSuccess) return cuda_fail(e, "ca_chunk_attention launch");
+  if (pl.persistent) {
+    e = launch_sk_combine(p, D, pl.NT, st);
+    if (e != cudaSuccess) return cuda_fail(e, "ca_chunk_attention combine launch");
+  }
   if (pl.n_splits > 1) {
     e = launch_split_combine(p.Opart, p.LSEpart, pl.n_splits, L, Hq, D, O, LSE, p.out_f32, st);
     if (e != cudaSuccess) return cuda_fail(e, "ca_chunk_attention combine launch");

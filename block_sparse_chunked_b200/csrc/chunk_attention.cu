@@ -67,10 +67,12 @@ struct Smem {
   static constexpr int kVOff = kKOff + kNS * kKV;
   static constexpr int kBarOff = kVOff + kNS * kKV;
   // barriers: q_full, full_k[NS], full_v[NS], empty_k[NS], empty_v[NS],
-  //           s_full[2], p_full[2], o_done, drain
-  static constexpr int kNumBars = 1 + 4 * kNS + 2 + 2 + 2;
+  //           s_full[2], p_full[2], o_done, drain, q_free
+  static constexpr int kNumBars = 1 + 4 * kNS + 2 + 2 + 3;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kMiscOff + 64;
+  // persistent schedule: per-unit live entries, prefix of stage counts, warp sums
+  static constexpr int kSchedOff = kMiscOff + 64;
+  static constexpr int kBytes = kSchedOff + (2 * 2048 + 1 + 32) * 4;
   static constexpr int kAlloc = kBytes + 1024;          // slack for 1024-B alignment
 };
 
@@ -87,6 +89,46 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, const A
   }
   return ok;
 }
+
+// Number of work units whose stage counts a persistent CTA keeps in shared memory.
+constexpr int kMaxUnits = 2048;
+
+// Unit u -> (group, 64-token query span, head slice); later query spans
+// (more causal blocks) first.
+struct UnitCoord {
+  int g, qs, hh;
+};
+__device__ __forceinline__ UnitCoord unit_coord(const AttnParams& p, int u) {
+  const int per_qs = p.Hkv * p.nhalves;
+  UnitCoord c;
+  c.qs = p.nqs - 1 - u / per_qs;
+  c.g = (u % per_qs) / p.nhalves;
+  c.hh = (u % per_qs) % p.nhalves;
+  return c;
+}
+
+// Live table entries of unit u: the entries <= its diagonal block, a prefix
+// of the ascending row (binary search).
+__device__ __forceinline__ int unit_live(const AttnParams& p, int u) {
+  const UnitCoord c = unit_coord(p, u);
+  const int diag_kb = p.nPblk + (c.qs * 64) / p.B;
+  const int32_t* trow = p.tables + (size_t)c.g * p.nKblk;
+  int cnt = p.counts[c.g];
+  if (cnt < 0 || cnt > p.nKblk) {
+    set_flag(p.err, CA_FLAG_BOUNDS);
+    cnt = cnt < 0 ? 0 : p.nKblk;
+  }
+  int lo = 0, hi = cnt;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (trow[mid] <= diag_kb) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// How a piece's result leaves the CTA.
+enum PieceOut : int { kOutFinal = 0, kOutSplit = 1, kOutSK = 2 };
 
 template <int D, int NT, bool QSPLIT>
 __global__ void __launch_bounds__(128 + NT * 128, 1)
@@ -111,48 +153,64 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
   auto p_full = [&](int t) { return bars + 8u * (3 + 4 * kNS + t); };
   const uint32_t o_done = bars + 8u * (5 + 4 * kNS);
   const uint32_t drain = bars + 8u * (6 + 4 * kNS);
+  const uint32_t q_free = bars + 8u * (7 + 4 * kNS);
   int* misc = reinterpret_cast<int*>(sm + S::kMiscOff);
-  // misc[0] tmem base, [1] n_live, [2] has_diag, [3] first stage, [4] stage count, [5] abort
+  // misc[0] tmem base, [1] live entries (one-piece mode), [2] first stage,
+  // [3] last stage (exclusive), [5] abort
   volatile int* abort_flag = misc + 5;
+  int* sk_live = reinterpret_cast<int*>(sm + S::kSchedOff);  // [kMaxUnits] (persistent)
+  int* sk_pref = sk_live + kMaxUnits;                         // [kMaxUnits + 1]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // ---- decode the work item (heaviest query spans first)
-  const int item = blockIdx.x;
-  const int split = item % p.n_splits;
-  const int unit = item / p.n_splits;
-  const int per_qs = p.Hkv * p.nhalves;
-  const int qs = p.nqs - 1 - unit / per_qs;
-  const int g = (unit % per_qs) / p.nhalves;
-  const int hh = (unit % per_qs) % p.nhalves;
-  const int t0 = qs * 64;
-  const int diag_kb = p.nPblk + t0 / p.B;
   const int spb = kStageKeys / p.B;  // pages per stage
-  const int32_t* trow = p.tables + (size_t)g * p.nKblk;
+  const int nthreads = 128 + NT * 128;
 
+  // ---- work: one piece (one-piece mode) or a contiguous range of all
+  // units' stages (persistent mode)
+  if (threadIdx.x == 0) misc[5] = 0;
+  if (!p.persistent) {
+    if (threadIdx.x == 0) {
+      const int u = blockIdx.x / p.n_splits, split = blockIdx.x % p.n_splits;
+      const int live = unit_live(p, u);
+      const int nst = (live + spb - 1) / spb;
+      misc[1] = live;
+      misc[2] = (int)((long long)split * nst / p.n_splits);
+      misc[3] = (int)((long long)(split + 1) * nst / p.n_splits);
+    }
+  } else {
+    // every CTA derives the same schedule: stage counts of all units, prefix sums
+    for (int u = threadIdx.x; u < p.n_units; u += nthreads) sk_live[u] = unit_live(p, u);
+    __syncthreads();
+    // block-wide exclusive scan of the stage counts: each thread a run of units
+    const int per = (p.n_units + nthreads - 1) / nthreads;
+    const int u0 = min(p.n_units, threadIdx.x * per), u1 = min(p.n_units, u0 + per);
+    int run = 0;
+    for (int u = u0; u < u1; ++u) run += (sk_live[u] + spb - 1) / spb;
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int* wsum = sk_pref + kMaxUnits + 1;  // scratch after the prefix array: [warps]
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += wsum[w];
+    int acc = base + incl - run;
+    for (int u = u0; u < u1; ++u) {
+      sk_pref[u] = acc;
+      acc += (sk_live[u] + spb - 1) / spb;
+    }
+    if (threadIdx.x == nthreads - 1) sk_pref[p.n_units] = base + incl;
+    __syncthreads();
+    if (blockIdx.x == 0)
+      for (int u = threadIdx.x; u <= p.n_units; u += nthreads) p.sk_sched[u] = sk_pref[u];
+  }
   if (threadIdx.x == 0) {
-    int cnt = p.counts[g];
-    if (cnt < 0 || cnt > p.nKblk) {
-      set_flag(p.err, CA_FLAG_BOUNDS);
-      cnt = cnt < 0 ? 0 : p.nKblk;
-    }
-    int lo = 0, hi = cnt;  // entries <= diag_kb form a prefix of the sorted row
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (trow[mid] <= diag_kb) lo = mid + 1;
-      else hi = mid;
-    }
-    const int n_live = lo;
-    const int nst = (n_live + spb - 1) / spb;
-    const int s0 = (int)((long long)split * nst / p.n_splits);
-    const int s1 = (int)((long long)(split + 1) * nst / p.n_splits);
-    misc[1] = n_live;
-    misc[2] = (n_live > 0 && trow[n_live - 1] == diag_kb) ? 1 : 0;
-    misc[3] = s0;
-    misc[4] = s1 - s0;
-    misc[5] = 0;
     mbar_init(q_full, 1);
+    mbar_init(q_free, 1);
     for (int s = 0; s < kNS; ++s) {
       mbar_init(full_k(s), 1);
       mbar_init(full_v(s), 1);
@@ -175,45 +233,79 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = (uint32_t)misc[0];
-  const int n_live = misc[1];
-  const int has_diag = misc[2];
-  const int s0 = misc[3];
-  const int nloc = misc[4];
-  const int nst_total = (n_live + spb - 1) / spb;
+
+  // Visit this CTA's pieces in order: fn(unit, live entries, first stage,
+  // end stage, output kind, partial slot).  Every role walks the same list.
+  auto for_each_piece = [&](auto&& fn) {
+    if (!p.persistent) {
+      const int split = blockIdx.x % p.n_splits;
+      fn(blockIdx.x / p.n_splits, misc[1], misc[2], misc[3],
+         p.n_splits > 1 ? kOutSplit : kOutFinal, split);
+      return;
+    }
+    const long long T = sk_pref[p.n_units];
+    const int P = p.sk_ctas, c = blockIdx.x;
+    // units without any stage: their rows are written by CTA (u mod P)
+    for (int u = c; u < p.n_units; u += P)
+      if (sk_pref[u + 1] == sk_pref[u]) fn(u, sk_live[u], 0, 0, kOutFinal, 0);
+    const int r0 = (int)(T * c / P), r1 = (int)(T * (c + 1) / P);
+    if (r1 <= r0) return;
+    int lo = 0, hi = p.n_units;  // first unit with pref[u + 1] > r0
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (sk_pref[mid + 1] > r0) hi = mid;
+      else lo = mid + 1;
+    }
+    bool first = true;
+    for (int u = lo; u < p.n_units && sk_pref[u] < r1; ++u) {
+      const int a = max(r0, sk_pref[u]) - sk_pref[u];
+      const int b = min(r1, sk_pref[u + 1]) - sk_pref[u];
+      if (b <= a) continue;
+      const bool whole = a == 0 && b == sk_pref[u + 1] - sk_pref[u];
+      fn(u, sk_live[u], a, b, whole ? kOutFinal : kOutSK, first ? 2 * c : 2 * c + 1);
+      first = false;
+    }
+  };
 
   if (warp == 0) {
     // ================================================================ producer
     // The whole warp runs the loop: lane i prefetches table entry i of the next
     // group of 32 and its page id, so the dependent lookups tables ->
-    // page_table are off the per-stage path; lane 0 issues the copies.
-    if (nloc > 0) {
-      const uint64_t pol = policy_evict_last();
-      if (lane == 0) {
-        prefetch_tmap(&tmQ);
-        if (QSPLIT) prefetch_tmap(&tmQlo);
-        prefetch_tmap(&tmK);
-        prefetch_tmap(&tmV);
+    // page_table are off the per-stage path; one elected lane issues copies.
+    const uint64_t pol = policy_evict_last();
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      if (QSPLIT) prefetch_tmap(&tmQlo);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+    }
+    int gj = 0, pn = 0;  // global stage counter, non-empty piece counter
+    bool ok = true;
+    for_each_piece([&](int u, int live, int s0, int s1, int, int) {
+      if (s1 <= s0 || !ok) return;
+      const UnitCoord uc = unit_coord(p, u);
+      const int32_t* trow = p.tables + (size_t)uc.g * p.nKblk;
+      if (pn > 0) ok = wait_warp(q_free, (pn - 1) & 1, p, abort_flag);
+      if (ok && lane == 0) {
         mbar_expect_tx(q_full, S::kQTerms * NT * 128 * D * 2);
         for (int q = 0; q < S::kQTerms; ++q)
           for (int t = 0; t < NT; ++t)
             for (int s = 0; s < 2; ++s) {
-              int hl = hh * p.HPU + 2 * t + s;  // head within the group
-              const int hcap = min(p.G - 1, hh * p.HPU + p.HPU - 1);
+              int hl = uc.hh * p.HPU + 2 * t + s;  // head within the group
+              const int hcap = min(p.G - 1, uc.hh * p.HPU + p.HPU - 1);
               hl = min(hl, hcap);
-              const int head = g * p.G + hl;
+              const int head = uc.g * p.G + hl;
               for (int c = 0; c < KCH; ++c)
                 tma_load_3d(sbase + S::kQOff + (q * NT + t) * S::kQTile + c * S::kChunkBytes +
                                 s * 64 * 128,
-                            q ? &tmQlo : &tmQ, q_full, c * 64, head, t0);
+                            q ? &tmQlo : &tmQ, q_full, c * 64, head, uc.qs * 64);
             }
       }
-      const int e_begin = s0 * spb;
-      const int e_end = min(n_live, (s0 + nloc) * spb);
+      const int e_begin = s0 * spb, e_end = min(live, s1 * spb);
       int pg_cache = 0, cache_base = -32;
-      bool ok = true;
-      for (int j = 0; j < nloc && ok; ++j) {
-        const int stage = s0 + j, slot = j % kNS, round = j / kNS;
-        const int npg = min(spb, n_live - stage * spb);
+      for (int stage = s0; stage < s1 && ok; ++stage, ++gj) {
+        const int slot = gj % kNS, round = gj / kNS;
+        const int npg = min(spb, live - stage * spb);
         const uint32_t bytes = (uint32_t)npg * p.B * D * 2;
         int page[2] = {0, 0};
         for (int pi = 0; pi < npg; ++pi) {
@@ -244,7 +336,7 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
           for (int pi = 0; pi < npg; ++pi)
             for (int c = 0; c < KCH; ++c)
               tma_load_4d_w(sbase + S::kKOff + slot * S::kKV + c * S::kChunkBytes + pi * p.B * 128,
-                            &tmK, full_k(slot), c * 64, 0, g, page[pi], pol);
+                            &tmK, full_k(slot), c * 64, 0, uc.g, page[pi], pol);
         }
         if (ok && round > 0) ok = wait_warp(empty_v(slot), (round - 1) & 1, p, abort_flag);
         if (ok) {
@@ -252,37 +344,43 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
           for (int pi = 0; pi < npg; ++pi)
             for (int c = 0; c < KCH; ++c)
               tma_load_4d_w(sbase + S::kVOff + slot * S::kKV + c * S::kChunkBytes + pi * p.B * 128,
-                            &tmV, full_v(slot), c * 64, 0, g, page[pi], pol);
+                            &tmV, full_v(slot), c * 64, 0, uc.g, page[pi], pol);
         }
       }
-      if (lane == 0) {
-        // Do not leave with copies in flight: the last stages' loads must land.
-        for (int j = max(0, nloc - kNS); j < nloc; ++j) {
-          mbar_wait(full_k(j % kNS), (j / kNS) & 1, p.wait_ns);
-          mbar_wait(full_v(j % kNS), (j / kNS) & 1, p.wait_ns);
-        }
+      ++pn;
+    });
+    if (lane == 0) {
+      // Do not leave with copies in flight: the last stages' loads must land.
+      for (int G = max(0, gj - kNS); G < gj; ++G) {
+        mbar_wait(full_k(G % kNS), (G / kNS) & 1, p.wait_ns);
+        mbar_wait(full_v(G % kNS), (G / kNS) & 1, p.wait_ns);
       }
+      if (pn > 0) mbar_wait(q_full, (pn - 1) & 1, p.wait_ns);
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
     // The whole warp runs this loop (addresses stay warp-uniform); one elected
     // lane issues each tcgen05.mma / commit.
-    if (nloc > 0) {
-      // Descriptors differ per MMA only in the start-address field (address >> 4
-      // in bits 0-13): build each operand's descriptor once and add the
-      // compile-time byte offset >> 4 per K-step.
-      constexpr uint32_t kIdescPV = idesc_bf16(128, D, 1);
-      constexpr uint32_t kIdescS128 = idesc_bf16(128, 128, 0);
-      constexpr uint32_t kIdescS64 = idesc_bf16(128, 64, 0);
-      uint64_t qdesc[NT];
+    // Descriptors differ per MMA only in the start-address field (address >> 4
+    // in bits 0-13): build each operand's descriptor once and add the
+    // compile-time byte offset >> 4 per K-step.
+    constexpr uint32_t kIdescPV = idesc_bf16(128, D, 1);
+    constexpr uint32_t kIdescS128 = idesc_bf16(128, 128, 0);
+    constexpr uint32_t kIdescS64 = idesc_bf16(128, 64, 0);
+    uint64_t qdesc[NT];
 #pragma unroll
-      for (int t = 0; t < NT; ++t) qdesc[t] = smem_desc_sw128(sbase + S::kQOff + t * S::kQTile, 16, 1024);
-      const uint64_t kdesc0 = smem_desc_sw128(sbase + S::kKOff, 16, 1024);
-      const uint64_t vdesc0 = smem_desc_sw128(sbase + S::kVOff, S::kChunkBytes, 1024);
-      auto npg_of = [&](int j) { return min(spb, n_live - (s0 + j) * spb); };
+    for (int t = 0; t < NT; ++t) qdesc[t] = smem_desc_sw128(sbase + S::kQOff + t * S::kQTile, 16, 1024);
+    const uint64_t kdesc0 = smem_desc_sw128(sbase + S::kKOff, 16, 1024);
+    const uint64_t vdesc0 = smem_desc_sw128(sbase + S::kVOff, S::kChunkBytes, 1024);
+    int gj = 0, pn = 0;
+    bool ok = true;
+    for_each_piece([&](int, int live, int s0, int s1, int, int) {
+      if (s1 <= s0 || !ok) return;
+      const int n = s1 - s0;
+      auto keys_of = [&](int j) { return min(spb, live - (s0 + j) * spb) * p.B; };
       auto issue_s = [&](int t, int j) {
-        const uint64_t kd = kdesc0 + (uint64_t)(((j % kNS) * S::kKV) >> 4);
-        const uint32_t idesc = npg_of(j) * p.B == 128 ? kIdescS128 : kIdescS64;
+        const uint64_t kd = kdesc0 + (uint64_t)((((gj + j) % kNS) * S::kKV) >> 4);
+        const uint32_t idesc = keys_of(j) == 128 ? kIdescS128 : kIdescS64;
         const uint32_t dt = tmem + 256 + t * 128;
 #pragma unroll
         for (int q = 0; q < S::kQTerms; ++q)
@@ -294,11 +392,11 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
           }
       };
       auto issue_pv = [&](int t, int j) {
-        const uint64_t vd = vdesc0 + (uint64_t)(((j % kNS) * S::kKV) >> 4);
+        const uint64_t vd = vdesc0 + (uint64_t)((((gj + j) % kNS) * S::kKV) >> 4);
         const uint32_t dt = tmem + t * 128;
         const uint32_t at = tmem + 256 + t * 128;
         const uint32_t acc0 = j > 0 ? 1u : 0u;
-        if (npg_of(j) * p.B == 128) {
+        if (keys_of(j) == 128) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts_w(dt, at + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), kIdescPV, kk > 0 ? 1u : acc0);
@@ -308,7 +406,8 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
             mma_ts_w(dt, at + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), kIdescPV, kk > 0 ? 1u : acc0);
         }
       };
-      bool ok = wait_warp(q_full, 0, p, abort_flag) && wait_warp(full_k(0), 0, p, abort_flag);
+      ok = wait_warp(q_full, pn & 1, p, abort_flag) &&
+           wait_warp(full_k(gj % kNS), (gj / kNS) & 1, p, abort_flag);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
@@ -317,25 +416,25 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
           issue_s(1, 0);
           mma_commit_w(s_full(1));
         }
-        mma_commit_w(empty_k(0));
+        mma_commit_w(empty_k(gj % kNS));
       }
-      for (int j = 0; j < nloc && ok; ++j) {
-        const int slot = j % kNS;
-        ok = wait_warp(p_full(0), j & 1, p, abort_flag) &&
-             wait_warp(full_v(slot), (j / kNS) & 1, p, abort_flag);
+      for (int j = 0; j < n && ok; ++j) {
+        const int G = gj + j, slot = G % kNS;
+        ok = wait_warp(p_full(0), G & 1, p, abort_flag) &&
+             wait_warp(full_v(slot), (G / kNS) & 1, p, abort_flag);
         if (!ok) break;
         tc_fence_after();
         issue_pv(0, j);
-        const bool more = j + 1 < nloc;
+        const bool more = j + 1 < n;
         if (more) {
-          ok = wait_warp(full_k((j + 1) % kNS), ((j + 1) / kNS) & 1, p, abort_flag);
+          ok = wait_warp(full_k((G + 1) % kNS), ((G + 1) / kNS) & 1, p, abort_flag);
           if (!ok) break;
           tc_fence_after();
           issue_s(0, j + 1);
           mma_commit_w(s_full(0));
         }
         if (NT == 2) {
-          ok = wait_warp(p_full(1), j & 1, p, abort_flag);
+          ok = wait_warp(p_full(1), G & 1, p, abort_flag);
           if (!ok) break;
           tc_fence_after();
           issue_pv(1, j);
@@ -346,151 +445,176 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
             issue_s(1, j + 1);
             mma_commit_w(s_full(1));
           }
-          mma_commit_w(empty_k((j + 1) % kNS));
+          mma_commit_w(empty_k((G + 1) % kNS));
         }
       }
-      if (ok) mma_commit_w(o_done);
-      // every MMA issued by this warp has finished before TMEM is released
-      mma_commit_w(drain);
-      mbar_wait(drain, 0, p.wait_ns);
-    }
+      if (ok) {
+        mma_commit_w(o_done);  // this piece's O is complete
+        mma_commit_w(q_free);  // and no MMA reads its Q any more
+      }
+      gj += n;
+      ++pn;
+    });
+    // every MMA issued by this warp has finished before TMEM is released
+    mma_commit_w(drain);
+    mbar_wait(drain, 0, p.wait_ns);
   } else if (warp >= 4) {
     // ================================================================ softmax / epilogue
     const int t = (warp - 4) >> 2;
     const int row = threadIdx.x & 127;
     const int sub = row >> 6;
-    const int tok = t0 + (row & 63);
-    const int hl_raw = hh * p.HPU + 2 * t + sub;
-    const bool valid_row = (2 * t + sub) < p.HPU && hl_raw < p.G;
-    const int head = g * p.G + min(hl_raw, p.G - 1);
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + 256 + t * 128;
     const uint32_t tO = tmem + lane_off + t * 128;
-    const int diag_lim = (t0 % p.B) + (row & 63);  // visible keys of the diagonal block: jl <= this
-    float m_used = -INFINITY, l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+    int gj = 0, pn = 0;
     bool ok = true;
-    for (int j = 0; j < nloc; ++j) {
-      const int stage = s0 + j;
-      const int npg = min(spb, n_live - stage * spb);
-      const int nvalid = npg * p.B;
-      const bool diag_stage = has_diag && (stage == nst_total - 1);
-      const int diag_c0 = (npg - 1) * p.B;  // first column of the diagonal page
-      ok = wait_warp(s_full(t), j & 1, p, abort_flag);
-      if (!ok) break;
-      tc_fence_after();
-      // One TMEM pass: the row's scores (raw Q.K) into registers.
-      float sr[kStageKeys];
-      tmem_ld64f(tS, sr);
-      if (nvalid > 64) tmem_ld64f(tS + 64, sr + 64);
-      tmem_wait_ld();
-      if (nvalid <= 64) {
+    for_each_piece([&](int u, int live, int s0, int s1, int out, int slot) {
+      const UnitCoord uc = unit_coord(p, u);
+      const int t0 = uc.qs * 64;
+      const int diag_kb = p.nPblk + t0 / p.B;
+      const int tok = t0 + (row & 63);
+      const int hl_raw = uc.hh * p.HPU + 2 * t + sub;
+      const bool valid_row = (2 * t + sub) < p.HPU && hl_raw < p.G;
+      const int head = uc.g * p.G + min(hl_raw, p.G - 1);
+      const int nst = (live + spb - 1) / spb;
+      const int32_t* trow = p.tables + (size_t)uc.g * p.nKblk;
+      const bool has_diag = live > 0 && trow[live - 1] == diag_kb;
+      const int diag_lim = (t0 % p.B) + (row & 63);  // visible keys of the diagonal block: jl <= this
+      const int n = s1 - s0;
+      float m_used = -INFINITY, l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+      for (int j = 0; j < n && ok; ++j) {
+        const int stage = s0 + j, G = gj + j;
+        const int npg = min(spb, live - stage * spb);
+        const int nvalid = npg * p.B;
+        const bool diag_stage = has_diag && (stage == nst - 1);
+        const int diag_c0 = (npg - 1) * p.B;  // first column of the diagonal page
+        ok = wait_warp(s_full(t), G & 1, p, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        // One TMEM pass: the row's scores (raw Q.K) into registers.
+        float sr[kStageKeys];
+        tmem_ld64f(tS, sr);
+        if (nvalid > 64) tmem_ld64f(tS + 64, sr + 64);
+        tmem_wait_ld();
+        if (nvalid <= 64) {
 #pragma unroll
-        for (int c = 64; c < kStageKeys; ++c) sr[c] = -INFINITY;
-      }
-      if (diag_stage) {  // token-level causal mask, diagonal block only
-#pragma unroll
-        for (int c = 0; c < kStageKeys; ++c)
-          if (c >= diag_c0 && (c - diag_c0) > diag_lim) sr[c] = -INFINITY;
-      }
-      // row max of the raw scores (scale > 0 commutes with max)
-      float mx0 = max3(sr[0], sr[1], sr[2]);
-      float mx1 = max3(sr[3], sr[4], sr[5]);
-#pragma unroll
-      for (int c = 6; c < kStageKeys - 2; c += 4) {
-        mx0 = max3(mx0, sr[c], sr[c + 1]);
-        mx1 = max3(mx1, sr[c + 2], sr[c + 3]);
-      }
-      const float mx = max3(mx0, mx1, fmaxf(sr[kStageKeys - 2], sr[kStageKeys - 1])) * p.scale_log2;
-      const float m_new = fmaxf(m_used, mx);
-      const bool need = (m_new != -INFINITY) && (m_new > m_used + 8.0f);
-      float alpha = 1.f;
-      if (need) {
-        alpha = ex2(m_used - m_new);  // 0 when m_used == -inf
-        l0 *= alpha;
-        l1 *= alpha;
-        l2 *= alpha;
-        l3 *= alpha;
-        m_used = m_new;
-      }
-      const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
-      const float sc = p.scale_log2;
-      // p = 2^(s*scale - m): packed FMA, then ex2; fp32 row sum before the bf16 rounding
-#pragma unroll
-      for (int c = 0; c < kStageKeys / 32; ++c) {
-        if (c * 32 < nvalid) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float x0, x1;
-            ffma2(x0, x1, sr[c * 32 + 2 * i], sr[c * 32 + 2 * i + 1], sc, sc, nm, nm);
-            const float e0 = ex2(x0), e1 = ex2(x1);
-            if (i & 1) fadd2(l2, l3, e0, e1);  // two independent sum chains
-            else fadd2(l0, l1, e0, e1);
-            pk[i] = pack_bf16x2(e0, e1);
-          }
-          tmem_st16(tS + c * 16, pk);
+          for (int c = 64; c < kStageKeys; ++c) sr[c] = -INFINITY;
         }
+        if (diag_stage) {  // token-level causal mask, diagonal block only
+#pragma unroll
+          for (int c = 0; c < kStageKeys; ++c)
+            if (c >= diag_c0 && (c - diag_c0) > diag_lim) sr[c] = -INFINITY;
+        }
+        // row max of the raw scores (scale > 0 commutes with max)
+        float mx0 = max3(sr[0], sr[1], sr[2]);
+        float mx1 = max3(sr[3], sr[4], sr[5]);
+#pragma unroll
+        for (int c = 6; c < kStageKeys - 2; c += 4) {
+          mx0 = max3(mx0, sr[c], sr[c + 1]);
+          mx1 = max3(mx1, sr[c + 2], sr[c + 3]);
+        }
+        const float mx = max3(mx0, mx1, fmaxf(sr[kStageKeys - 2], sr[kStageKeys - 1])) * p.scale_log2;
+        const float m_new = fmaxf(m_used, mx);
+        const bool need = (m_new != -INFINITY) && (m_new > m_used + 8.0f);
+        float alpha = 1.f;
+        if (need) {
+          alpha = ex2(m_used - m_new);  // 0 when m_used == -inf
+          l0 *= alpha;
+          l1 *= alpha;
+          l2 *= alpha;
+          l3 *= alpha;
+          m_used = m_new;
+        }
+        const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
+        const float sc = p.scale_log2;
+        // p = 2^(s*scale - m): packed FMA, then ex2; fp32 row sum before the bf16 rounding
+#pragma unroll
+        for (int c = 0; c < kStageKeys / 32; ++c) {
+          if (c * 32 < nvalid) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float x0, x1;
+              ffma2(x0, x1, sr[c * 32 + 2 * i], sr[c * 32 + 2 * i + 1], sc, sc, nm, nm);
+              const float e0 = ex2(x0), e1 = ex2(x1);
+              if (i & 1) fadd2(l2, l3, e0, e1);  // two independent sum chains
+              else fadd2(l0, l1, e0, e1);
+              pk[i] = pack_bf16x2(e0, e1);
+            }
+            tmem_st16(tS + c * 16, pk);
+          }
+        }
+        // O still holds the sum over earlier stages at the old max: bring it to the new one
+        if (__any_sync(0xffffffffu, need) && j > 0) {
+          uint32_t r[32];
+          for (int c = 0; c < D / 32; ++c) {
+            tmem_ld32(tO + c * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(tO + c * 32, r);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full(t));
       }
-      // O still holds the sum over earlier stages at the old max: bring it to the new one
-      if (__any_sync(0xffffffffu, need) && j > 0) {
-        uint32_t r[32];
-        for (int c = 0; c < D / 32; ++c) {
+      // ---- epilogue of the piece
+      const bool ran = ok && n > 0;
+      bool have_o = false;
+      if (ran) {
+        have_o = wait_warp(o_done, pn & 1, p, abort_flag);
+        ok = have_o;
+        if (have_o) tc_fence_after();
+      }
+      const float l = (l0 + l1) + (l2 + l3);
+      const bool have = have_o && l > 0.f;
+      const float inv = have ? 1.f / l : 0.f;
+      const float lse = have ? (m_used + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      uint32_t r[32];
+      for (int c = 0; c < D / 32; ++c) {
+        if (have_o) {
           tmem_ld32(tO + c * 32, r);
           tmem_wait_ld();
+        } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(tO + c * 32, r);
+          for (int i = 0; i < 32; ++i) r[i] = 0u;
         }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full(t));
-    }
-    // ---- epilogue
-    const float l = (l0 + l1) + (l2 + l3);
-    if (ok && nloc > 0) ok = wait_warp(o_done, 0, p, abort_flag);
-    if (ok && nloc > 0) tc_fence_after();
-    const bool have = ok && nloc > 0 && l > 0.f;
-    const float inv = have ? 1.f / l : 0.f;
-    const float lse = have ? (m_used + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
-    const bool split_out = p.n_splits > 1;
-    uint32_t r[32];
-    for (int c = 0; c < D / 32; ++c) {
-      if (ok && nloc > 0) {
-        tmem_ld32(tO + c * 32, r);
-        tmem_wait_ld();
-      } else {
+        if (!valid_row) continue;
+        float v[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = 0u;
-      }
-      if (!valid_row) continue;
-      float v[32];
+        for (int i = 0; i < 32; ++i) v[i] = have ? __uint_as_float(r[i]) * inv : 0.f;
+        float* fdst = nullptr;
+        if (out == kOutSplit)
+          fdst = p.Opart + (((size_t)slot * p.L + tok) * p.Hq + head) * D + c * 32;
+        else if (out == kOutSK)
+          fdst = p.Osk + ((size_t)slot * (NT * 128) + t * 128 + row) * D + c * 32;
+        else if (p.out_f32)
+          fdst = reinterpret_cast<float*>(p.O) + ((size_t)tok * p.Hq + head) * D + c * 32;
+        if (fdst) {
+          float4* dst = reinterpret_cast<float4*>(fdst);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = have ? __uint_as_float(r[i]) * inv : 0.f;
-      if (split_out) {
-        float4* dst = reinterpret_cast<float4*>(
-            p.Opart + (((size_t)split * p.L + tok) * p.Hq + head) * D + c * 32);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-      } else if (p.out_f32) {
-        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.O) +
+          for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.O) +
                                                 ((size_t)tok * p.Hq + head) * D + c * 32);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-      } else {
-        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.O) +
-                                              ((size_t)tok * p.Hq + head) * D + c * 32);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          dst[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
-                              pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                                pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+        }
       }
-    }
-    if (valid_row) {
-      if (split_out) p.LSEpart[((size_t)split * p.Hq + head) * p.L + tok] = lse;
-      else p.LSE[(size_t)head * p.L + tok] = lse;
-    }
+      if (valid_row) {
+        if (out == kOutSplit) p.LSEpart[((size_t)slot * p.Hq + head) * p.L + tok] = lse;
+        else if (out == kOutSK) p.LSEsk[(size_t)slot * (NT * 128) + t * 128 + row] = lse;
+        else p.LSE[(size_t)head * p.L + tok] = lse;
+      }
+      if (n > 0) {
+        gj += n;
+        ++pn;
+      }
+    });
     tc_fence_before();
   }
   __syncthreads();
@@ -498,6 +622,65 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// Persistent mode: merge the pieces of every unit that more than one CTA
+// worked on.  Block (u, r8) handles rows [8*r8, 8*r8 + 8) of unit u, one warp
+// per row (lane = D/32 consecutive columns, coalesced).  The pieces sit in
+// consecutive CTAs of the stage ranges, and their partial slots follow from
+// the same schedule the attention kernel used.
+template <int D, int NT>
+__global__ void __launch_bounds__(256)
+    sk_combine_kernel(const AttnParams p) {
+  const int u = blockIdx.x;
+  const int32_t* pref = p.sk_sched;
+  const long long T = pref[p.n_units];
+  const int P = p.sk_ctas;
+  const long long a = pref[u], b = pref[u + 1];
+  if (b <= a) return;  // no stage: written by the attention kernel
+  auto cta_of = [&](long long s) { return (int)(((s + 1) * P - 1) / T); };
+  auto cta_start = [&](int c) { return (T * c) / P; };
+  const int ca = cta_of(a), cb = cta_of(b - 1);
+  if (ca == cb) return;  // one CTA did the whole unit and wrote it
+  const int r = blockIdx.y * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  const UnitCoord uc = unit_coord(p, u);
+  const int t = r >> 7, sub = (r >> 6) & 1;
+  const int tok = uc.qs * 64 + (r & 63);
+  const int hl_raw = uc.hh * p.HPU + 2 * t + sub;
+  if (!((2 * t + sub) < p.HPU && hl_raw < p.G)) return;
+  const int head = uc.g * p.G + hl_raw;
+  auto slot_of = [&](int c) { return (c == ca && cta_start(c) < a) ? 2 * c + 1 : 2 * c; };
+  float m = -INFINITY;
+  for (int c = ca; c <= cb; ++c) m = fmaxf(m, p.LSEsk[(size_t)slot_of(c) * (NT * 128) + r]);
+  constexpr int PER = D / 32;
+  float acc[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+  float tot = 0.f;
+  if (m != -INFINITY) {
+    for (int c = ca; c <= cb; ++c) {
+      const int sl = slot_of(c);
+      const float ls = p.LSEsk[(size_t)sl * (NT * 128) + r];
+      if (ls == -INFINITY) continue;
+      const float w = __expf(ls - m);
+      tot += w;
+      const float* src = p.Osk + ((size_t)sl * (NT * 128) + r) * D + lane * PER;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) acc[i] += w * src[i];
+    }
+  }
+  const float inv = tot > 0.f ? 1.f / tot : 0.f;
+  const size_t o = ((size_t)tok * p.Hq + head) * D + lane * PER;
+  if (p.out_f32) {
+#pragma unroll
+    for (int i = 0; i < PER; ++i) reinterpret_cast<float*>(p.O)[o + i] = acc[i] * inv;
+  } else {
+#pragma unroll
+    for (int i = 0; i < PER; i += 2)
+      *reinterpret_cast<uint32_t*>(reinterpret_cast<__nv_bfloat16*>(p.O) + o + i) =
+          pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
+  }
+  if (lane == 0) p.LSE[(size_t)head * p.L + tok] = tot > 0.f ? m + __logf(tot) : -INFINITY;
 }
 
 // Merge the fp32 partials of a KV-range split by their LSE.
@@ -616,6 +799,16 @@ cudaError_t launch_chunk_attention(const CUtensorMap& q, const CUtensorMap& qlo,
   CA_LAUNCH(64, 1, true)
 #undef CA_LAUNCH
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_sk_combine(const AttnParams& p, int D, int NT, cudaStream_t st) {
+  const dim3 grid(p.n_units, NT * 128 / 8);
+  if (D == 128 && NT == 2) sk_combine_kernel<128, 2><<<grid, 256, 0, st>>>(p);
+  else if (D == 128 && NT == 1) sk_combine_kernel<128, 1><<<grid, 256, 0, st>>>(p);
+  else if (D == 64 && NT == 2) sk_combine_kernel<64, 2><<<grid, 256, 0, st>>>(p);
+  else if (D == 64 && NT == 1) sk_combine_kernel<64, 1><<<grid, 256, 0, st>>>(p);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
 }
 
 cudaError_t launch_split_combine(const float* Opart, const float* LSEpart, int n_splits, int L,

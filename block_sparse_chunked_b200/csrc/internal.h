@@ -18,6 +18,12 @@ struct AttnParams {
   float* Opart;      // [S, L, Hq, D] fp32      (n_splits > 1)
   float* LSEpart;    // [S, Hq, L] fp32         (n_splits > 1)
   int32_t* err;      // device error word (may be null)
+  // persistent (stream-K) mode: each of sk_ctas CTAs takes an equal range of
+  // all units' KV stages; split units leave fp32 partials for sk_combine
+  int32_t* sk_sched;  // [n_units + 1] prefix of per-unit stage counts (written by CTA 0)
+  float* Osk;         // [2 * sk_ctas][NT*128][D]
+  float* LSEsk;       // [2 * sk_ctas][NT*128]
+  int persistent, n_units, sk_ctas;
   int Hq, Hkv, G, HPU, nhalves, L, P, B, nPblk, nKblk, num_pages, n_splits, nqs, out_f32;
   float scale_log2;  // log2(e) / sqrt(D)
   unsigned long long wait_ns;
@@ -29,6 +35,7 @@ cudaError_t launch_chunk_attention(const CUtensorMap& q, const CUtensorMap& qlo,
                                    const CUtensorMap& k, const CUtensorMap& v,
                                    const AttnParams& p, int D, int NT, bool qsplit, int grid,
                                    cudaStream_t st);
+cudaError_t launch_sk_combine(const AttnParams& p, int D, int NT, cudaStream_t st);
 cudaError_t launch_split_combine(const float* Opart, const float* LSEpart, int n_splits, int L,
                                  int Hq, int D, void* O, float* LSE, int out_f32,
                                  cudaStream_t st);

@@ -79,10 +79,10 @@ int ca_build_tables_batched(const uint8_t* masks, int nb, int Hq, int Hkv, int n
 
 /*
  * ca_workspace_size — bytes of device workspace ca_chunk_attention needs for
- * these shapes: bf16 copies of fp32 inputs (dtype == CA_DTYPE_FP32) and the
- * fp32 partial results of a KV-range split (n_splits > 1; n_splits <= 0
- * means the split ca_chunk_attention picks by itself).  Returns 0 when none
- * is needed, and (size_t)-1 for invalid shapes.
+ * these shapes: bf16 copies of fp32 inputs (dtype == CA_DTYPE_FP32), the
+ * schedule and fp32 partial results of the automatic persistent mode
+ * (n_splits <= 0), or the fp32 partials of a KV-range split (n_splits > 1).
+ * Returns 0 when none is needed, and (size_t)-1 for invalid shapes.
  */
 size_t ca_workspace_size(int dtype, int Hq, int Hkv, int head_dim, int block, int chunk_len,
                          int prefix_len, int num_pages, int n_splits);
@@ -113,7 +113,12 @@ size_t ca_workspace_size(int dtype, int Hq, int Hkv, int head_dim, int block, in
  *   O           [L, Hq, d] (out), dtype `dtype`
  *   LSE         float32 [Hq, L] (out), natural log
  *   workspace   >= ca_workspace_size(...) bytes (may be NULL if that is 0)
- *   n_splits    KV-range splits per work unit (<= 0: automatic)
+ *   n_splits    <= 0: automatic — one CTA per unit when there are at least
+ *               as many units (group x 64-token span x head slice) as SMs;
+ *               otherwise a persistent grid of at most one CTA per SM splits
+ *               all units' KV stages evenly and merges the pieces of split
+ *               units by LSE (needs workspace); 1: one CTA per unit; k > 1:
+ *               each unit's KV range split k ways, merged by LSE
  *   err_flag    int32 (device, may be NULL): the kernels OR CA_FLAG_* into it
  *               on an out-of-range table entry / page id (the access is
  *               clamped, results are then undefined) or on a pipeline wait

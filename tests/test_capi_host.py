@@ -76,7 +76,7 @@ def _attn(bsc, **kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(Q=None), -1), (dict(dtype=7), -3), (dict(P=1000), -2), (dict(L=100), -2),
     (dict(B=32), -1), (dict(d=96), -1), (dict(Hq=6, Hkv=4), -1), (dict(num_pages=19), -1),
-    (dict(Q=ctypes.c_void_p(0x1001)), -1), (dict(dtype=1), -7), (dict(S=4), -7),
+    (dict(Q=ctypes.c_void_p(0x1001)), -1), (dict(dtype=1), -7), (dict(S=4), -7), (dict(S=0), -7),
 ])
 def test_chunk_attention_rejects_bad_arguments(bsc, kw, code):
     assert _attn(bsc, **kw) == code
@@ -85,8 +85,14 @@ def test_chunk_attention_rejects_bad_arguments(bsc, kw, code):
 
 def test_workspace_size_rules(bsc):
     ws = bsc.lib.ca_workspace_size
-    # bf16, >= one CTA per SM of units: no split, no workspace
+    # bf16, one CTA per unit: no workspace
+    assert ws(0, 32, 8, 128, 64, 2048, 129024, 2048, 1) == 0
+    # automatic mode, 256 units >= 148 SMs: one CTA per unit, no workspace
     assert ws(0, 32, 8, 128, 64, 2048, 129024, 2048, 0) == 0
+    # automatic mode, 16 units: persistent grid of min(148, 16*12/4) = 48 CTAs,
+    # schedule + fp32 partials of <= 2 pieces per CTA
+    n = ws(0, 8, 2, 128, 64, 512, 1024, 24, 0)
+    assert 2 * 48 * 256 * 128 * 4 <= n < 2 * 48 * 256 * 130 * 4 + 65536
     # explicit split: fp32 partials + LSE partials
     n = ws(0, 32, 8, 128, 64, 2048, 129024, 2048, 2)
     assert n >= 2 * 2048 * 32 * 128 * 4 + 2 * 32 * 2048 * 4

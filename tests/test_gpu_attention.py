@@ -86,7 +86,7 @@ MEDIUM = [
 
 
 @pytest.mark.parametrize("Hq,Hkv,d,B,P,L,kind,rho", MEDIUM)
-@pytest.mark.parametrize("n_splits", [1, 3])
+@pytest.mark.parametrize("n_splits", [0, 1, 3])
 def test_medium_cases_full(bsc, Hq, Hkv, d, B, P, L, kind, rho, n_splits):
     w = workloads.Workload("m", Hq, Hkv, d, "bf16", P, L, B, kind, rho=rho, corr=0.5,
                            window=4, seed=Hq + P + L + B)
