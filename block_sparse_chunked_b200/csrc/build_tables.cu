@@ -25,8 +25,22 @@ namespace cg = cooperative_groups;
 
 namespace ca {
 
+#ifndef CA_BUILD_CTAS_PER_SM
+#define CA_BUILD_CTAS_PER_SM 2
+#endif
+#ifndef CA_BUILD_UNROLL
+#define CA_BUILD_UNROLL 8
+#endif
 constexpr int kBuildThreads = 256;
+constexpr int kRowUnroll = CA_BUILD_UNROLL;
 constexpr int kMaxSlab = 8192;  // columns per CTA -> 256 bit-set words, one per thread
+
+// Streaming (evict-first) loads: each mask byte is read exactly once.
+__device__ __forceinline__ uint4 ldcs(const uint4* p) { return __ldcs(p); }
+__device__ __forceinline__ uint32_t ldcs(const uint32_t* p) { return __ldcs(p); }
+__device__ __forceinline__ uint8_t ldcs(const uint8_t* p) {
+  return (uint8_t)__ldcs(reinterpret_cast<const unsigned char*>(p));
+}
 
 template <int VEC>
 struct VecLoad;
@@ -105,9 +119,9 @@ __global__ void __launch_bounds__(kBuildThreads)
       const T* p = reinterpret_cast<const T*>(base + (size_t)rt * nKblk + c0) + v;
       const size_t step = (size_t)RT * nKblk / VEC;
       int r = rt;
-#pragma unroll 8
+#pragma unroll kRowUnroll
       for (; r < R; r += RT) {
-        V::orin(acc, __ldg(p));
+        V::orin(acc, ldcs(p));  // read once: stream past L2
         p += step;
       }
     }
@@ -178,8 +192,13 @@ template __global__ void build_tables_kernel<1>(const uint8_t*, int, int, int, i
 cudaError_t launch_build_tables(const uint8_t* mask, int nb, int Hq, int Hkv, int nQblk,
                                 int nKblk, int32_t* tables, int32_t* counts,
                                 cudaStream_t stream) {
-  int C = (nKblk + 255) / 256;  // ~256+ columns per CTA
-  if (C > 8) C = 8;
+  // Cluster size: enough CTAs for ~CA_BUILD_CTAS_PER_SM per SM over all (mask, group) units,
+  // at most 8 per cluster and at least 256 columns per CTA.
+  const long long units = (long long)nb * Hkv;
+  int C = (int)((CA_BUILD_CTAS_PER_SM * 148 + units - 1) / units);
+  C = C > 8 ? 8 : C;
+  const int cmax = (nKblk + 255) / 256;
+  C = C > cmax ? cmax : C;
   if (C < 1) C = 1;
   int slab = (nKblk + C - 1) / C;
   slab = (slab + 31) & ~31;
