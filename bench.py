@@ -109,6 +109,16 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise max of a list of floats over all ranks (the device times
+    of a step are reported as the slowest rank's)."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 def make_sets(w, nsets, dev):
     """nsets input sets on the device: distinct page buffers (same values, distinct
     addresses) and masks drawn with seeds 0..nsets-1."""
@@ -315,10 +325,7 @@ def main():
     mean_step = statistics.mean(step_ms)
     mean_attn = statistics.mean(attn_ms)
     mean_flops = statistics.mean(flops)
-    tot = torch.tensor([mean_step, mean_attn], dtype=torch.float64, device=dev)
-    if pg:
-        pg.all_reduce(tot, op=pg.ReduceOp.MAX)
-    mean_step, mean_attn = float(tot[0]), float(tot[1])
+    mean_step, mean_attn = max_over_ranks([mean_step, mean_attn], pg, dev)
     value = world * mean_flops / (mean_step * 1e-3) / 1e12
     attn_tflops = mean_flops / (mean_attn * 1e-3) / 1e12
 
@@ -407,10 +414,8 @@ def main():
     e2e_flops = bsc.selected_flops(sets[0]["tables"].cpu().numpy(),
                                    sets[0]["counts"].cpu().numpy(), w.Hq, w.nPblk, w.nQblk,
                                    w.block, w.head_dim)
-    e2e_t = torch.tensor([statistics.mean(e2e_ms)], dtype=torch.float64, device=dev)
-    if pg:
-        pg.all_reduce(e2e_t, op=pg.ReduceOp.MAX)
-    e2e_value = world * e2e_flops / (float(e2e_t[0]) * 1e-3) / 1e12
+    e2e_mean = max_over_ranks([statistics.mean(e2e_ms)], pg, dev)[0]
+    e2e_value = world * e2e_flops / (e2e_mean * 1e-3) / 1e12
 
     if rank == 0:
         peak = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
@@ -441,7 +446,7 @@ def main():
                          "per_launch": "selected FLOPs of one 2048-token chunk (32 heads)",
                          "traffic": None},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
-                    "d2h_bytes_per_step": int(d2h), "ms_per_step": float(e2e_t[0])},
+                    "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_mean},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
         }
