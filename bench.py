@@ -375,6 +375,31 @@ def main():
         bt.append(a.elapsed_time(b))
     bbytes = bsc.builder_bytes(nb, w.Hq, w.Hkv, w.nQblk, w.nKblk)
     build_gbs = bbytes / (statistics.mean(bt) * 1e-3) / 1e9
+    # the same union from bit-packed masks (one bit per block), 32 and 128 masks per launch
+    bits_res = {}
+    for nbb in (32, 128):
+        nrot = 4 if nbb == 32 else 2
+        bb = [torch.from_numpy(wl.pack_mask_bits(np.stack([wl.mask_for(w, seed=300 + nbb * r + k)
+                                                           for k in range(nbb)])).view(np.int32))
+              .to(dev) for r in range(nrot)]
+        tbb = torch.empty(nbb, w.Hkv, w.nKblk, dtype=torch.int32, device=dev)
+        cbb = torch.empty(nbb, w.Hkv, dtype=torch.int32, device=dev)
+        for r in range(nrot):
+            bsc.build_tables_bits(bb[r], w.Hkv, w.nKblk, tbb, cbb)
+        tt = []
+        for r in range(12):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            bsc.build_tables_bits(bb[r % nrot], w.Hkv, w.nKblk, tbb, cbb)
+            b.record(stream)
+            torch.cuda.synchronize()
+            tt.append(a.elapsed_time(b))
+        nbytes = bsc.builder_bytes(nbb, w.Hq, w.Hkv, w.nQblk, w.nKblk, bits=True)
+        gbs = nbytes / (statistics.mean(tt) * 1e-3) / 1e9
+        bits_res[str(nbb)] = {"us": statistics.mean(tt) * 1e3, "GB/s": gbs,
+                              "frac_of_measured_hbm": gbs / peaks.get("hbm_gbs", 1.0),
+                              "mask_bytes_per_mask": w.Hq * w.nQblk * 4 * ((w.nKblk + 31) // 32)}
+        del bb
     single_bytes = bsc.builder_bytes(1, w.Hq, w.Hkv, w.nQblk, w.nKblk)
 
     # ---- end to end through the public API with pinned host buffers
@@ -436,6 +461,7 @@ def main():
             "table_build_single_gbs": single_bytes / (statistics.mean(build_ms) * 1e-3) / 1e9,
             "dense_ms": dense_ms_mean, "dense_tflops": dense_flops / (dense_ms_mean * 1e-3) / 1e12,
             "speedup_vs_dense": dense_ms_mean / mean_attn,
+            "table_build_bits": bits_res,
             "table_build_batched": {"masks_per_launch": nb, "us": statistics.mean(bt) * 1e3,
                                     "GB/s": build_gbs, "frac_of_measured_hbm": build_gbs / hbm,
                                     "frac_of_8TBs_nominal": build_gbs / 8000.0},

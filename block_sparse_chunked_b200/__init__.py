@@ -23,6 +23,7 @@ from ._capi import (  # noqa: F401
     version,
     build_tables,
     build_tables_batched,
+    build_tables_bits,
     workspace_size,
     chunk_attention,
     check,

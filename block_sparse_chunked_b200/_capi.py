@@ -25,6 +25,7 @@ EXPORTS = {
     "ca_build_tables": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "ca_build_tables_batched": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp,
                                          _vp]),
+    "ca_build_tables_bits": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "ca_workspace_size": (_c_size, [_c_int] * 9),
     "ca_chunk_attention": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _vp, _c_int, _c_int,
                                     _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _c_size,
@@ -118,6 +119,22 @@ def build_tables(mask, Hkv, tables=None, counts=None):
     if counts is None:
         counts = torch.empty(Hkv, dtype=torch.int32, device=mask.device)
     _ok(lib.ca_build_tables(_ptr(mask), Hq, Hkv, nQ, nK, _ptr(tables), _ptr(counts), _stream()))
+    return tables, counts
+
+
+def build_tables_bits(mask_bits, Hkv, nKblk, tables=None, counts=None):
+    """Bit-packed masks int32/uint32 [nb, Hq, nQblk, ceil(nKblk/32)] (bit j of word w selects
+    block 32w + j) -> tables int32 [nb, Hkv, nKblk], counts int32 [nb, Hkv]."""
+    _need_cuda("mask_bits", mask_bits, (torch.int32, torch.uint32), 4)
+    nb, Hq, nQ, W = mask_bits.shape
+    if W != (nKblk + 31) // 32:
+        raise ValueError(f"mask_bits has {W} words per row, nKblk={nKblk} needs {(nKblk + 31) // 32}")
+    if tables is None:
+        tables = torch.empty(nb, Hkv, nKblk, dtype=torch.int32, device=mask_bits.device)
+    if counts is None:
+        counts = torch.empty(nb, Hkv, dtype=torch.int32, device=mask_bits.device)
+    _ok(lib.ca_build_tables_bits(_ptr(mask_bits), nb, Hq, Hkv, nQ, nKblk, _ptr(tables),
+                                 _ptr(counts), _stream()))
     return tables, counts
 
 

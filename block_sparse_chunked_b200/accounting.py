@@ -35,6 +35,8 @@ def dense_flops(Hq, nPblk, nQblk, block, head_dim):
     return 4.0 * block * block * head_dim * dense_pairs(Hq, nPblk, nQblk)
 
 
-def builder_bytes(nb, Hq, Hkv, nQblk, nKblk):
-    """Algorithmic bytes of one table-builder launch: mask read + tables + counts written."""
-    return nb * (Hq * nQblk * nKblk + Hkv * nKblk * 4 + Hkv * 4)
+def builder_bytes(nb, Hq, Hkv, nQblk, nKblk, bits=False):
+    """Algorithmic bytes of one table-builder launch: mask read (one byte per block, or
+    one bit packed in 32-bit words) + tables + counts written."""
+    mask = Hq * nQblk * (4 * ((nKblk + 31) // 32) if bits else nKblk)
+    return nb * (mask + Hkv * nKblk * 4 + Hkv * 4)

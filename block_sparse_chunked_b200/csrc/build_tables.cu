@@ -232,3 +232,120 @@ cudaError_t launch_build_tables(const uint8_t* mask, int nb, int Hq, int Hkv, in
 }
 
 }  // namespace ca
+
+namespace ca {
+
+// ---------------------------------------------------------------------------
+// Bit-packed masks: bit j of 32-bit word w of a row selects KV block 32w + j.
+// The union of a group is a word-wise OR over its G*nQblk rows (8x fewer bytes
+// than one byte per block); one CTA per (mask, group) ORs the rows with 16-
+// or 4-byte loads, then ranks the set bits with a block scan of per-thread
+// popcounts and writes the ascending entries and the -1 padding.
+constexpr int kBitsThreads = 256;
+constexpr int kMaxBitWords = 2048;  // nKblk <= 65536
+
+template <int VECW>  // words per load: 4 (uint4) or 1
+__global__ void __launch_bounds__(kBitsThreads)
+    build_tables_bits_kernel(const uint32_t* __restrict__ bits, int Hq, int Hkv, int nQblk,
+                             int nKblk, int32_t* __restrict__ tables,
+                             int32_t* __restrict__ counts) {
+  __shared__ uint32_t uni[kMaxBitWords];
+  __shared__ int warp_sum[kBitsThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int G = Hq / Hkv, R = G * nQblk;
+  const int W = (nKblk + 31) >> 5;
+  const uint32_t* base = bits + ((size_t)b * Hq + (size_t)g * G) * (size_t)nQblk * W;
+  for (int w = tid; w < W; w += kBitsThreads) uni[w] = 0u;
+  __syncthreads();
+
+  // ---- OR down the group's rows
+  const int nv = W / VECW;
+  int CW = 1;
+  while (CW < nv && CW < kBitsThreads) CW <<= 1;
+  const int RT = kBitsThreads / CW, rt = tid / CW;
+  for (int v = tid % CW; v < nv; v += CW) {
+    if (VECW == 4) {
+      uint4 acc = make_uint4(0, 0, 0, 0);
+      const uint4* p = reinterpret_cast<const uint4*>(base + (size_t)rt * W) + v;
+      const size_t step = (size_t)RT * W / 4;
+#pragma unroll 8
+      for (int r = rt; r < R; r += RT) {
+        const uint4 x = __ldcs(p);
+        acc.x |= x.x; acc.y |= x.y; acc.z |= x.z; acc.w |= x.w;
+        p += step;
+      }
+      if (acc.x) atomicOr(&uni[4 * v], acc.x);
+      if (acc.y) atomicOr(&uni[4 * v + 1], acc.y);
+      if (acc.z) atomicOr(&uni[4 * v + 2], acc.z);
+      if (acc.w) atomicOr(&uni[4 * v + 3], acc.w);
+    } else {
+      uint32_t acc = 0u;
+      const uint32_t* p = base + (size_t)rt * W + v;
+      const size_t step = (size_t)RT * W;
+#pragma unroll 8
+      for (int r = rt; r < R; r += RT) {
+        acc |= __ldcs(p);
+        p += step;
+      }
+      if (acc) atomicOr(&uni[v], acc);
+    }
+  }
+  __syncthreads();
+  if (tid == 0 && (nKblk & 31)) uni[W - 1] &= (1u << (nKblk & 31)) - 1u;  // bits past nKblk
+  __syncthreads();
+
+  // ---- rank: thread t owns words [t*k, t*k + k)
+  const int k = (W + kBitsThreads - 1) / kBitsThreads;
+  const int w0 = min(W, tid * k), w1 = min(W, w0 + k);
+  int cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(uni[w]);
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sum[warp] = incl;
+  __syncthreads();
+  int before = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < kBitsThreads / 32; ++w) {
+    before += (w < warp) ? warp_sum[w] : 0;
+    total += warp_sum[w];
+  }
+  int pos = before + incl - cnt;
+  int32_t* trow = tables + ((size_t)b * Hkv + g) * nKblk;
+  for (int w = w0; w < w1; ++w) {
+    uint32_t x = uni[w];
+    while (x) {
+      const int bit = __ffs(x) - 1;
+      trow[pos++] = w * 32 + bit;
+      x &= x - 1;
+    }
+  }
+  for (int q = total + tid; q < nKblk; q += kBitsThreads) trow[q] = -1;
+  if (tid == 0) counts[(size_t)b * Hkv + g] = total;
+}
+
+template __global__ void build_tables_bits_kernel<4>(const uint32_t*, int, int, int, int, int32_t*,
+                                                     int32_t*);
+template __global__ void build_tables_bits_kernel<1>(const uint32_t*, int, int, int, int, int32_t*,
+                                                     int32_t*);
+
+cudaError_t launch_build_tables_bits(const uint32_t* bits, int nb, int Hq, int Hkv, int nQblk,
+                                     int nKblk, int32_t* tables, int32_t* counts,
+                                     cudaStream_t stream) {
+  const int W = (nKblk + 31) / 32;
+  if (W > kMaxBitWords) return cudaErrorInvalidValue;
+  const dim3 grid(Hkv, nb);
+  if (W % 4 == 0 && (reinterpret_cast<uintptr_t>(bits) & 15u) == 0)
+    build_tables_bits_kernel<4><<<grid, kBitsThreads, 0, stream>>>(bits, Hq, Hkv, nQblk, nKblk,
+                                                                   tables, counts);
+  else
+    build_tables_bits_kernel<1><<<grid, kBitsThreads, 0, stream>>>(bits, Hq, Hkv, nQblk, nKblk,
+                                                                   tables, counts);
+  return cudaGetLastError();
+}
+
+}  // namespace ca

@@ -192,6 +192,25 @@ int ca_build_tables(const uint8_t* mask, int Hq, int Hkv, int nQblk, int nKblk, 
   return ca_build_tables_batched(mask, 1, Hq, Hkv, nQblk, nKblk, tables, counts, stream);
 }
 
+int ca_build_tables_bits(const uint32_t* mask_bits, int nb, int Hq, int Hkv, int nQblk,
+                         int nKblk, int32_t* tables, int32_t* counts, void* stream) {
+  if (!mask_bits || !tables || !counts) return fail(CA_ERR_ARG, "ca_build_tables_bits: null pointer");
+  if (nb < 1 || nb > 65535)
+    return fail(CA_ERR_ARG, "ca_build_tables_bits: nb=%d out of [1,65535]", nb);
+  if (Hq < 1 || Hkv < 1 || Hkv > Hq || Hq % Hkv || Hkv > 65535)
+    return fail(CA_ERR_ARG, "ca_build_tables_bits: Hq=%d must be a positive multiple of Hkv=%d",
+                Hq, Hkv);
+  if (nQblk < 1) return fail(CA_ERR_ARG, "ca_build_tables_bits: nQblk=%d < 1", nQblk);
+  if (nKblk < 1 || nKblk > 65536)
+    return fail(CA_ERR_ARG, "ca_build_tables_bits: nKblk=%d out of [1,65536]", nKblk);
+  if (reinterpret_cast<uintptr_t>(mask_bits) & 3u)
+    return fail(CA_ERR_ARG, "ca_build_tables_bits: mask_bits must be 4-byte aligned");
+  cudaError_t e = launch_build_tables_bits(mask_bits, nb, Hq, Hkv, nQblk, nKblk, tables, counts,
+                                           static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "ca_build_tables_bits launch");
+  return CA_OK;
+}
+
 size_t ca_workspace_size(int dtype, int Hq, int Hkv, int head_dim, int block, int chunk_len,
                          int prefix_len, int num_pages, int n_splits) {
   Plan pl;

@@ -31,6 +31,9 @@ struct AttnParams {
 
 cudaError_t launch_build_tables(const uint8_t* mask, int nb, int Hq, int Hkv, int nQblk,
                                 int nKblk, int32_t* tables, int32_t* counts, cudaStream_t stream);
+cudaError_t launch_build_tables_bits(const uint32_t* bits, int nb, int Hq, int Hkv, int nQblk,
+                                     int nKblk, int32_t* tables, int32_t* counts,
+                                     cudaStream_t stream);
 cudaError_t launch_chunk_attention(const CUtensorMap& q, const CUtensorMap& qlo,
                                    const CUtensorMap& k, const CUtensorMap& v,
                                    const AttnParams& p, int D, int NT, bool qsplit, int grid,

@@ -78,6 +78,22 @@ int ca_build_tables_batched(const uint8_t* masks, int nb, int Hq, int Hkv, int n
                             int nKblk, int32_t* tables, int32_t* counts, void* stream);
 
 /*
+ * ca_build_tables_bits — the same union and tables from bit-packed masks
+ * (one bit per (head, Q-block, KV block) instead of one byte: 8x less to
+ * read).  Same method ("CompactAttention ...", Abstract: Q-block union and
+ * intra-group union into minimal per-group KV block tables).
+ *
+ *   mask_bits  uint32 [nb, Hq, nQblk, W], W = ceil(nKblk / 32): bit j (least
+ *              significant first) of word w of row (h, qb) selects KV block
+ *              32w + j; bits at or past nKblk in the last word are ignored.
+ *              4-byte aligned (16-byte alignment with W % 4 == 0 is faster).
+ *   tables, counts  as for ca_build_tables_batched.
+ * Limits: 1 <= nb <= 65535, Hq % Hkv == 0, nQblk >= 1, 1 <= nKblk <= 65536.
+ */
+int ca_build_tables_bits(const uint32_t* mask_bits, int nb, int Hq, int Hkv, int nQblk,
+                         int nKblk, int32_t* tables, int32_t* counts, void* stream);
+
+/*
  * ca_workspace_size — bytes of device workspace ca_chunk_attention needs for
  * these shapes: bf16 copies of fp32 inputs (dtype == CA_DTYPE_FP32), the
  * schedule and fp32 partial results of the automatic persistent mode

@@ -22,7 +22,7 @@ Every function here is pinned by tests/test_oracle_*.py against brute force,
 closed forms, library routines (torch SDPA in float64) and invariants.
 Nothing here is "parity unpinned".
 """
-from .tables import oracle_tables, brute_force_tables  # noqa: F401
+from .tables import oracle_tables, brute_force_tables, unpack_mask_bits, oracle_tables_bits  # noqa: F401
 from .attention import (  # noqa: F401
     depage,
     oracle_chunk_attention,

@@ -48,3 +48,18 @@ def brute_force_tables(mask, Hkv):
         counts[g] = len(s)
         tables[g][:len(s)] = s
     return np.array(tables, dtype=np.int32), np.array(counts, dtype=np.int32)
+
+
+def unpack_mask_bits(bits, nKblk):
+    """uint32 words [..., W] -> uint8 mask [..., nKblk]: block kb is bit (kb mod 32),
+    least significant first, of word kb // 32; bits at or past nKblk are ignored."""
+    words = np.asarray(bits, dtype=np.uint32)
+    out = np.zeros(words.shape[:-1] + (nKblk,), dtype=np.uint8)
+    for kb in range(nKblk):
+        out[..., kb] = (words[..., kb // 32] >> np.uint32(kb % 32)) & np.uint32(1)
+    return out
+
+
+def oracle_tables_bits(bits, Hkv, nKblk):
+    """Tables from bit-packed masks: the same set definition on the unpacked mask."""
+    return oracle_tables(unpack_mask_bits(bits, nKblk), Hkv)

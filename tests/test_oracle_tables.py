@@ -136,3 +136,23 @@ def test_planted_dropped_group_head_is_caught(monkeypatch):
     tw, cw = wrong(m, 2)
     tb, cb = oracle.brute_force_tables(m.tolist(), 2)
     assert not (np.array_equal(tw, tb) and np.array_equal(cw, cb))
+
+
+def test_unpack_bits_hand_example():
+    """Word 0x00000005 selects blocks 0 and 2; word 1 bit 1 (0x2) selects block 33;
+    a set bit past nKblk = 35 (block 34+) is ignored."""
+    bits = np.array([[[0x00000005, 0x00000002 | 0x00000008]]], dtype=np.uint32)  # bit 3 of w1 = block 35
+    m = oracle.unpack_mask_bits(bits, 35)
+    assert np.flatnonzero(m[0, 0]).tolist() == [0, 2, 33]
+
+
+@pytest.mark.parametrize("nK", [1, 31, 32, 33, 100, 2048])
+def test_pack_unpack_roundtrip(nK):
+    rng = np.random.default_rng(nK)
+    m = (rng.random((3, 2, nK)) < 0.3).astype(np.uint8)
+    bits = workloads.pack_mask_bits(m)
+    assert bits.shape == (3, 2, (nK + 31) // 32) and bits.dtype == np.uint32
+    assert np.array_equal(oracle.unpack_mask_bits(bits, nK), m)
+    t1, c1 = oracle.oracle_tables_bits(bits, 1, nK)
+    t2, c2 = oracle.oracle_tables(m, 1)
+    assert np.array_equal(t1, t2) and np.array_equal(c1, c2)

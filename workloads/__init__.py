@@ -11,6 +11,7 @@ from .generators import (  # noqa: F401
     bernoulli_mask,
     vertical_slash_mask,
     ones_mask,
+    pack_mask_bits,
     mask_for,
     causal_live,
 )

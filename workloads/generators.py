@@ -103,3 +103,14 @@ def mask_for(w, seed=None, clip=True):
     if w.mask_kind == "ones":
         return ones_mask(w.Hq, w.nPblk, w.nQblk, w.nKblk)
     raise ValueError(w.mask_kind)
+
+
+def pack_mask_bits(mask):
+    """uint8 mask [..., nKblk] -> uint32 words [..., ceil(nKblk/32)], bit j of word w
+    (least significant first) = mask[..., 32w + j] != 0; bits past nKblk are 0."""
+    m = (np.asarray(mask) != 0)
+    nK = m.shape[-1]
+    W = (nK + 31) // 32
+    pad = np.zeros(m.shape[:-1] + (W * 32 - nK,), dtype=bool)
+    b = np.packbits(np.concatenate([m, pad], axis=-1), axis=-1, bitorder="little")
+    return np.ascontiguousarray(b).view("<u4").astype(np.uint32)
