@@ -13,8 +13,9 @@ never finds the previous step's selected pages in L2.
 
 value = selected-block FLOPs per step / device time per step (TFLOP/s);
 e2e   = the same metric through the public API with pinned host buffers:
-        H2D of the mask, Q, the chunk's own K/V pages and the page table,
-        build + attention, D2H of O and LSE, all inside the timed region.
+        H2D of the mask, Q, the chunk's new K/V rows and the page table,
+        KV append into the paged cache + build + attention, D2H of O and LSE,
+        all inside the timed region.
 Also reported: the density-100% path on the same shapes (attention speedup),
 the batched table builder in GB/s (32 masks per launch), roofline fractions
 against the measured peaks, and the float64 oracle timed on host cores.
@@ -138,6 +139,19 @@ def make_sets(w, nsets, dev):
              "LSE": torch.empty(w.Hq, w.chunk_len, dtype=torch.float32, device=dev)}
         sets.append(d)
     return x, sets
+
+
+def timed_launch(stream, fn):
+    """Device time (ms) of the launches fn() makes.  A sleep kernel keeps the
+    GPU busy while the host enqueues them, so the host-side call overhead of a
+    lone launch does not land between the two events."""
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(200_000)  # ~0.1 ms at the B200's clocks
+    a.record(stream)
+    fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
 
 
 def run_step(bsc, w, s, ws, err):
@@ -267,14 +281,11 @@ def main():
         tb = torch.empty(nb, w.Hkv, w.nKblk, dtype=torch.int32, device=dev)
         cb = torch.empty(nb, w.Hkv, dtype=torch.int32, device=dev)
         ts = []
+        stream = torch.cuda.current_stream()
         for i in range(args.warmup + args.steps):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            bsc.build_tables_batched(masks, w.Hkv, tb, cb)
-            b.record()
-            torch.cuda.synchronize()
+            t_ = timed_launch(stream, lambda: bsc.build_tables_batched(masks, w.Hkv, tb, cb))
             if i >= args.warmup:
-                ts.append(a.elapsed_time(b))
+                ts.append(t_)
         nbytes = bsc.builder_bytes(nb, w.Hq, w.Hkv, w.nQblk, w.nKblk)
         print(json.dumps({"builder_masks": nb, "bytes": nbytes, "us": statistics.mean(ts) * 1e3,
                           "GB/s": nbytes / (statistics.mean(ts) * 1e-3) / 1e9}), flush=True)
@@ -344,14 +355,11 @@ def main():
     dense_ms = []
     for i in range(2 + 4):
         s = sets[i % len(sets)]
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        bsc.chunk_attention(s["Q"], s["K"], s["V"], s["pt"], dense_t, dense_c, w.prefix_len,
-                            err_flag=err, out=s["O"], lse=s["LSE"], workspace=ws)
-        b.record(stream)
-        torch.cuda.synchronize()
+        t_ = timed_launch(stream, lambda: bsc.chunk_attention(
+            s["Q"], s["K"], s["V"], s["pt"], dense_t, dense_c, w.prefix_len, err_flag=err,
+            out=s["O"], lse=s["LSE"], workspace=ws))
         if i >= 2:
-            dense_ms.append(a.elapsed_time(b))
+            dense_ms.append(t_)
     bsc.check(err)
     dense_flops = bsc.dense_flops(w.Hq, w.nPblk, w.nQblk, w.block, w.head_dim)
     dense_ms_mean = statistics.mean(dense_ms)
@@ -367,12 +375,7 @@ def main():
         bsc.build_tables_batched(mb[r], w.Hkv, tb, cb)
     bt = []
     for r in range(12):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        bsc.build_tables_batched(mb[r % 4], w.Hkv, tb, cb)
-        b.record(stream)
-        torch.cuda.synchronize()
-        bt.append(a.elapsed_time(b))
+        bt.append(timed_launch(stream, lambda: bsc.build_tables_batched(mb[r % 4], w.Hkv, tb, cb)))
     bbytes = bsc.builder_bytes(nb, w.Hq, w.Hkv, w.nQblk, w.nKblk)
     build_gbs = bbytes / (statistics.mean(bt) * 1e-3) / 1e9
     # the same union from bit-packed masks (one bit per block), 32 and 128 masks per launch
@@ -388,12 +391,8 @@ def main():
             bsc.build_tables_bits(bb[r], w.Hkv, w.nKblk, tbb, cbb)
         tt = []
         for r in range(12):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            bsc.build_tables_bits(bb[r % nrot], w.Hkv, w.nKblk, tbb, cbb)
-            b.record(stream)
-            torch.cuda.synchronize()
-            tt.append(a.elapsed_time(b))
+            tt.append(timed_launch(stream, lambda: bsc.build_tables_bits(bb[r % nrot], w.Hkv,
+                                                                        w.nKblk, tbb, cbb)))
         nbytes = bsc.builder_bytes(nbb, w.Hq, w.Hkv, w.nQblk, w.nKblk, bits=True)
         gbs = nbytes / (statistics.mean(tt) * 1e-3) / 1e9
         bits_res[str(nbb)] = {"us": statistics.mean(tt) * 1e3, "GB/s": gbs,
@@ -408,11 +407,17 @@ def main():
     h_q = x["Q"].pin_memory()
     h_pt = x["page_table"].pin_memory()
     pt_np = x["page_table"].numpy()
-    h_kc = x["K_pages"][torch.from_numpy(pt_np[chunk_blocks]).long()].contiguous().pin_memory()
-    h_vc = x["V_pages"][torch.from_numpy(pt_np[chunk_blocks]).long()].contiguous().pin_memory()
+    chunk_pages = torch.from_numpy(pt_np[chunk_blocks]).long()
+
+    def chunk_rows(pages):  # the chunk's own keys (values) as [L, Hkv, d] rows
+        return (pages[chunk_pages].permute(0, 2, 1, 3)
+                .reshape(w.chunk_len, w.Hkv, w.head_dim).contiguous().pin_memory())
+
+    h_kn, h_vn = chunk_rows(x["K_pages"]), chunk_rows(x["V_pages"])
+    d_kn, d_vn = torch.empty_like(h_kn, device=dev), torch.empty_like(h_vn, device=dev)
     h_o = torch.empty(w.chunk_len, w.Hq, w.head_dim, dtype=torch.bfloat16).pin_memory()
     h_l = torch.empty(w.Hq, w.chunk_len, dtype=torch.float32).pin_memory()
-    h2d = (h_mask.numel() + h_q.numel() * 2 + h_pt.numel() * 4 + h_kc.numel() * 2 * 2)
+    h2d = (h_mask.numel() + h_q.numel() * 2 + h_pt.numel() * 4 + h_kn.numel() * 2 * 2)
     d2h = h_o.numel() * 2 + h_l.numel() * 4
     e2e_ms = []
     for i in range(args.warmup + args.steps):
@@ -422,10 +427,9 @@ def main():
         s["mask"].copy_(h_mask, non_blocking=True)
         s["Q"].copy_(h_q, non_blocking=True)
         s["pt"].copy_(h_pt, non_blocking=True)
-        for j, kb in enumerate(chunk_blocks):
-            page = int(pt_np[kb])
-            s["K"][page].copy_(h_kc[j], non_blocking=True)
-            s["V"][page].copy_(h_vc[j], non_blocking=True)
+        d_kn.copy_(h_kn, non_blocking=True)
+        d_vn.copy_(h_vn, non_blocking=True)
+        bsc.append_kv(d_kn, d_vn, s["K"], s["V"], s["pt"], w.prefix_len, err_flag=err)
         bsc.build_tables(s["mask"], w.Hkv, s["tables"], s["counts"])
         bsc.chunk_attention(s["Q"], s["K"], s["V"], s["pt"], s["tables"], s["counts"],
                             w.prefix_len, err_flag=err, out=s["O"], lse=s["LSE"], workspace=ws)
@@ -436,6 +440,19 @@ def main():
         if i >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
     bsc.check(err)
+    # ---- the KV append kernel alone (chunk rows already resident)
+    ta = []
+    for r in range(12):
+        s = sets[r % len(sets)]
+        t_ = timed_launch(stream, lambda: bsc.append_kv(d_kn, d_vn, s["K"], s["V"], s["pt"],
+                                                        w.prefix_len, err_flag=err))
+        if r >= 4:
+            ta.append(t_)
+    bsc.check(err)
+    append_bytes = 2 * 2 * d_kn.numel() * d_kn.element_size()   # K and V, read once + written once
+    append_res = {"us": statistics.mean(ta) * 1e3,
+                  "GB/s": append_bytes / (statistics.mean(ta) * 1e-3) / 1e9,
+                  "bytes_per_launch": append_bytes}
     e2e_flops = bsc.selected_flops(sets[0]["tables"].cpu().numpy(),
                                    sets[0]["counts"].cpu().numpy(), w.Hq, w.nPblk, w.nQblk,
                                    w.block, w.head_dim)
@@ -462,6 +479,7 @@ def main():
             "dense_ms": dense_ms_mean, "dense_tflops": dense_flops / (dense_ms_mean * 1e-3) / 1e12,
             "speedup_vs_dense": dense_ms_mean / mean_attn,
             "table_build_bits": bits_res,
+            "kv_append": append_res,
             "table_build_batched": {"masks_per_launch": nb, "us": statistics.mean(bt) * 1e3,
                                     "GB/s": build_gbs, "frac_of_measured_hbm": build_gbs / hbm,
                                     "frac_of_8TBs_nominal": build_gbs / 8000.0},

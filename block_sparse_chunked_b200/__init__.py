@@ -26,6 +26,7 @@ from ._capi import (  # noqa: F401
     build_tables_bits,
     workspace_size,
     chunk_attention,
+    append_kv,
     check,
     wait_probe,
     last_error,

@@ -34,6 +34,8 @@ EXPORTS = {
                                             _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int,
                                             _vp, _vp]),
     "ca_noalloc_scratch_bytes": (_c_size, []),
+    "ca_append_kv": (_c_int, [_vp, _vp, _c_int, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int,
+                              _c_int, _c_int, _vp, _vp]),
     "ca_check": (_c_int, [_vp, _vp]),
     "ca_wait_probe": (_c_int, [_vp, _c_int, _vp]),
     "ca_last_error": (_c_int, [ctypes.c_char_p, _c_size]),
@@ -187,6 +189,22 @@ def chunk_attention(Q, K_pages, V_pages, page_table, tables, counts, prefix_len,
         _ptr(counts), Hq, Hkv, d, B, L, prefix_len, _ptr(out), _ptr(lse),
         _ptr(workspace) if ws_n else None, ws_n, n_splits, _ptr(err_flag), _stream()))
     return out, lse
+
+
+def append_kv(K_new, V_new, K_pages, V_pages, page_table, prefix_len, err_flag=None):
+    """Write the chunk's K_new/V_new [L, Hkv, d] into their pages (in place)."""
+    _need_cuda("K_new", K_new, tuple(_DT), 3)
+    _need_cuda("V_new", V_new, (K_new.dtype,), 3)
+    _need_cuda("K_pages", K_pages, (K_new.dtype,), 4)
+    _need_cuda("V_pages", V_pages, (K_new.dtype,), 4)
+    _need_cuda("page_table", page_table, (torch.int32,), 1)
+    L, Hkv, d = K_new.shape
+    num_pages, Hkv2, B, d2 = K_pages.shape
+    if V_new.shape != K_new.shape or V_pages.shape != K_pages.shape or Hkv2 != Hkv or d2 != d:
+        raise ValueError("append_kv: inconsistent shapes")
+    _ok(lib.ca_append_kv(_ptr(K_new), _ptr(V_new), _DT[K_new.dtype], _ptr(K_pages), _ptr(V_pages),
+                         num_pages, _ptr(page_table), Hkv, d, B, prefix_len, L, _ptr(err_flag),
+                         _stream()))
 
 
 def check(err_flag):

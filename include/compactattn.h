@@ -185,6 +185,25 @@ int ca_chunk_attention_noalloc(const void* Q, const void* K_pages, const void* V
 size_t ca_noalloc_scratch_bytes(void);
 
 /*
+ * ca_append_kv — write a prefill chunk's new keys and values into the paged
+ * KV cache in place, before ca_chunk_attention reads them ("CompactAttention
+ * ...", Abstract: chunked prefill over an accumulated, paged KV cache).
+ *
+ * Token i of the chunk (position p = prefix_len + i) goes to
+ * K_pages[page_table[p / B], g, p % B, :] = K_new[i, g, :] (V alike).
+ *   K_new, V_new      [chunk_len, Hkv, head_dim], dtype `dtype`
+ *   K_pages, V_pages  [num_pages, Hkv, B, head_dim], same dtype (written)
+ *   page_table        int32 [ceil((prefix_len + chunk_len) / B)]
+ * prefix_len need not be a multiple of B; chunk_len may be 0 (then K_new and
+ * V_new may be NULL and nothing is launched).  head_dim * element size must be a
+ * multiple of 16 bytes; buffers 16-byte aligned.  A page id out of range sets
+ * CA_FLAG_BOUNDS in *err_flag (may be NULL) and that row is skipped.
+ */
+int ca_append_kv(const void* K_new, const void* V_new, int dtype, void* K_pages, void* V_pages,
+                 int num_pages, const int32_t* page_table, int Hkv, int head_dim, int block,
+                 int prefix_len, int chunk_len, int32_t* err_flag, void* stream);
+
+/*
  * ca_check — synchronise `stream`, read *err_flag (device int32), clear it,
  * and map it to CA_OK / CA_ERR_BOUNDS / CA_ERR_TIMEOUT.
  */

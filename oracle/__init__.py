@@ -29,4 +29,5 @@ from .attention import (  # noqa: F401
     oracle_rows,
     brute_force_attention,
     lse_combine,
+    oracle_append_kv,
 )

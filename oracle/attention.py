@@ -173,3 +173,23 @@ def lse_combine(O_parts, LSE_parts):
     scale = np.where(live, 1.0, 0.0)[None] * np.exp(LSE_parts - np.where(live, LSE, 0.0)[None])
     O = (scale[..., None] * O_parts).sum(axis=0)
     return O, LSE
+
+
+def oracle_append_kv(K_pages, V_pages, page_table, K_new, V_new, prefix_len):
+    """Writing a chunk into the paged cache: token i of the chunk, at position
+    p = prefix_len + i, lands in row p mod B of page page_table[p // B].
+
+    Works on numpy arrays or torch CPU tensors (any dtype: a pure copy) and
+    returns updated copies of the two page arrays.
+    """
+    def _copy(x):
+        return x.clone() if hasattr(x, "clone") else np.array(x, copy=True)
+
+    K, V = _copy(K_pages), _copy(V_pages)
+    B = K.shape[2]
+    for i in range(K_new.shape[0]):
+        p = prefix_len + i
+        page = int(page_table[p // B])
+        K[page, :, p % B, :] = K_new[i]
+        V[page, :, p % B, :] = V_new[i]
+    return K, V

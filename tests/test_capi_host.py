@@ -109,3 +109,21 @@ def test_check_and_probe_reject_null(bsc):
 def test_accounting_dense_128k(bsc):
     # 32 heads x sum_{qb<32} (2016 + qb + 1) pairs x 4 * 64^2 * 128 FLOPs
     assert bsc.dense_flops(32, 2016, 32, 64, 128) == 4 * 64 * 64 * 128 * 32 * (32 * 2017 + 496)
+
+
+def _append(bsc, **kw):
+    a = dict(K=FAKE, V=FAKE, dtype=0, KP=FAKE, VP=FAKE, num_pages=40, pt=FAKE, Hkv=2, d=128, B=64,
+             P=100, L=64, err=None)
+    a.update(kw)
+    return bsc.lib.ca_append_kv(a["K"], a["V"], a["dtype"], a["KP"], a["VP"], a["num_pages"],
+                                a["pt"], a["Hkv"], a["d"], a["B"], a["P"], a["L"], a["err"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(K=None), -1), (dict(pt=None), -1), (dict(dtype=5), -3), (dict(d=4), -1),
+    (dict(d=6, dtype=1), -1), (dict(Hkv=0), -1), (dict(P=-1), -1), (dict(B=0), -1),
+    (dict(num_pages=2), -1), (dict(KP=ctypes.c_void_p(0x1008)), -1),
+])
+def test_append_kv_rejects_bad_arguments(bsc, kw, code):
+    assert _append(bsc, **kw) == code
+    assert "ca_append_kv" in bsc.last_error()
