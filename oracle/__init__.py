@@ -30,4 +30,5 @@ from .attention import (  # noqa: F401
     brute_force_attention,
     lse_combine,
     oracle_append_kv,
+    oracle_varlen,
 )

@@ -70,7 +70,7 @@ def oracle_chunk_attention(Q, K_pages, V_pages, page_table, tables, counts, pref
     Q = np.asarray(Q, dtype=np.float64)
     L_c, Hq, d = Q.shape
     Hkv, B = np.asarray(K_pages).shape[1], np.asarray(K_pages).shape[2]
-    nKblk = (prefix_len + L_c) // B
+    nKblk = -(-(prefix_len + L_c) // B)  # blocks holding positions 0 .. P + L_c - 1
     G = Hq // Hkv
     K = depage(K_pages, page_table, nKblk)
     V = depage(V_pages, page_table, nKblk)
@@ -86,6 +86,33 @@ def oracle_chunk_attention(Q, K_pages, V_pages, page_table, tables, counts, pref
             o, lse = _attend(Q[i0:i1, h, :], Kj, Vj, J, pos, d)
             O[i0:i1, h, :] = o
             LSE[h, i0:i1] = lse
+    return O, LSE
+
+
+def oracle_varlen(Q, K_pages, V_pages, cu_q, prefix_len, page_table, cu_pages, tables, counts):
+    """A batch of sequences sharing one page pool: sequence s has chunk rows
+    cu_q[s] .. cu_q[s+1] of Q, prefix prefix_len[s], page table
+    page_table[cu_pages[s] ...] and tables [Hkv, nKblk_s] stored flat from
+    Hkv * cu_pages[s]; each is exactly the single-sequence definition.
+    Returns O [total_q, Hq, d] and LSE [Hq, total_q]."""
+    Q = np.asarray(Q, dtype=np.float64)
+    total_q, Hq, d = Q.shape
+    Hkv, B = np.asarray(K_pages).shape[1], np.asarray(K_pages).shape[2]
+    tables = np.asarray(tables)
+    counts = np.asarray(counts).reshape(-1, Hkv)
+    O = np.zeros((total_q, Hq, d))
+    LSE = np.full((Hq, total_q), -np.inf)
+    for s in range(len(prefix_len)):
+        q0, q1, P = int(cu_q[s]), int(cu_q[s + 1]), int(prefix_len[s])
+        if q1 == q0:
+            continue
+        nK = -(-(P + q1 - q0) // B)
+        p0 = int(cu_pages[s])
+        pt = np.asarray(page_table)[p0:p0 + nK]
+        tab = tables[Hkv * p0:Hkv * p0 + Hkv * nK].reshape(Hkv, nK)
+        o, lse = oracle_chunk_attention(Q[q0:q1], K_pages, V_pages, pt, tab, counts[s], P)
+        O[q0:q1] = o
+        LSE[:, q0:q1] = lse
     return O, LSE
 
 
@@ -177,7 +204,9 @@ def lse_combine(O_parts, LSE_parts):
 
 def oracle_append_kv(K_pages, V_pages, page_table, K_new, V_new, prefix_len):
     """Writing a chunk into the paged cache: token i of the chunk, at position
-    p = prefix_len + i, lands in row p mod B of page page_table[p // B].
+    p = prefix_len + i, lands in row p mod B of page page_table[p // B]; the
+    rows of that last block after the chunk's last position are cleared to 0
+    (empty slots of the sequence's last block).
 
     Works on numpy arrays or torch CPU tensors (any dtype: a pure copy) and
     returns updated copies of the two page arrays.
@@ -187,9 +216,16 @@ def oracle_append_kv(K_pages, V_pages, page_table, K_new, V_new, prefix_len):
 
     K, V = _copy(K_pages), _copy(V_pages)
     B = K.shape[2]
-    for i in range(K_new.shape[0]):
+    L = K_new.shape[0]
+    for i in range(L):
         p = prefix_len + i
         page = int(page_table[p // B])
         K[page, :, p % B, :] = K_new[i]
         V[page, :, p % B, :] = V_new[i]
+    if L > 0:
+        last = prefix_len + L - 1
+        page = int(page_table[last // B])
+        for r in range(last % B + 1, B):
+            K[page, :, r, :] = 0
+            V[page, :, r, :] = 0
     return K, V

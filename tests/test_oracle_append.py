@@ -46,8 +46,21 @@ def test_readback_through_depage(prefix, L, B):
     # pages outside the table are untouched
     other = np.setdiff1d(np.arange(num_pages), pt)
     assert np.array_equal(K2[other], K[other]) and np.array_equal(V2[other], V[other])
-    # exactly L rows per head changed (values are distinct with probability 1)
-    assert int((K2 != K).any(axis=-1).sum()) == L * Hkv
+    # the rest of the last block is cleared; exactly L + tail rows per head changed
+    tail = (B - (prefix + L) % B) % B if L else 0
+    if tail:
+        seqK0 = oracle.depage(K2, pt, nK)
+        assert np.all(seqK0[:, prefix + L:prefix + L + tail] == 0)
+    assert int((K2 != K).any(axis=-1).sum()) == (L + tail) * Hkv
+
+
+def test_hand_placed_tail_is_cleared():
+    # B = 4, one page; prefix 1, chunk 2: positions 1, 2 written, position 3 cleared,
+    # position 0 (the prefix) kept.
+    K = np.full((1, 1, 4, 1), 7.0)
+    K2, _ = oracle.oracle_append_kv(K, K, [0], np.array([[[1.0]], [[2.0]]]),
+                                    np.array([[[1.0]], [[2.0]]]), 1)
+    assert K2[0, 0, :, 0].tolist() == [7.0, 1.0, 2.0, 0.0]
 
 
 def test_planted_off_by_one_is_caught():

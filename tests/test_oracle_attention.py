@@ -288,3 +288,103 @@ def test_planted_dropped_key_is_caught(monkeypatch):
     Or, Lr = sdpa_reference(Q, oracle.depage(Kp, pt, w.nKblk), oracle.depage(Vp, pt, w.nKblk),
                             vis, w.G)
     assert np.abs(L - Lr).max() > 1e-6
+
+
+# ---- unaligned prefix / chunk lengths and batches of sequences
+
+def unaligned_case(seed, Hq=4, Hkv=2, d=16, B=8, P=21, Lc=13, rho=0.3):
+    w = workloads.Workload("u", Hq, Hkv, d, "fp32", P, Lc, B, "bernoulli", rho=rho, seed=seed)
+    x = workloads.make_qkv_pages(w)
+    m = workloads.mask_for(w)
+    t, c = oracle.oracle_tables(m, Hkv)
+    return w, x, m, t, c
+
+
+@pytest.mark.parametrize("P,Lc", [(21, 13), (0, 5), (7, 1), (8, 9), (3, 30)])
+def test_unaligned_token_masked_sdpa(P, Lc):
+    w, x, m, t, c = unaligned_case(seed=P + Lc, P=P, Lc=Lc)
+    assert w.nKblk == -(-(P + Lc) // w.block)
+    Q, Kp, Vp = _np(x["Q"]), _np(x["K_pages"]), _np(x["V_pages"])
+    pt = x["page_table"].numpy()
+    O, L = oracle.oracle_chunk_attention(Q, Kp, Vp, pt, t, c, P)
+    Kf, Vf = oracle.depage(Kp, pt, w.nKblk), oracle.depage(Vp, pt, w.nKblk)
+    vis = token_visibility(t, c, w.Hq, w.Hkv, P, Lc, w.block, w.nKblk)
+    Or, Lr = sdpa_reference(Q, Kf, Vf, vis, w.G)
+    np.testing.assert_allclose(O, Or, rtol=0, atol=1e-10)
+    np.testing.assert_allclose(L, Lr, rtol=0, atol=1e-10)
+
+
+def test_unaligned_brute_force():
+    w, x, m, t, c = unaligned_case(seed=3, Hq=2, Hkv=1, d=4, B=4, P=6, Lc=5)
+    args = (_np(x["Q"]), _np(x["K_pages"]), _np(x["V_pages"]), x["page_table"].numpy(), t, c, 6)
+    O, L = oracle.oracle_chunk_attention(*args)
+    Ob, Lb = oracle.brute_force_attention(args[0].tolist(), args[1].tolist(), args[2].tolist(),
+                                          *args[3:])
+    np.testing.assert_allclose(O, Ob, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(L, Lb, rtol=0, atol=1e-12)
+
+
+def test_unaligned_masks_select_the_last_live_block():
+    """Q-block qb of a chunk at prefix P reaches block (P + last token of qb) // B."""
+    last = workloads.last_live_block(21, 13, 8)        # Q-blocks: tokens 0-7, 8-12
+    assert last.tolist() == [(21 + 7) // 8, (21 + 12) // 8]
+    live = workloads.causal_live(0, 2, 5, last)
+    assert live.sum(axis=1).tolist() == [4, 5]
+
+
+def test_unaligned_chunk_composition_equals_one_shot_causal():
+    """All-ones masks over chunks of ragged lengths reproduce full causal attention."""
+    Hq, Hkv, d, B = 4, 2, 16, 8
+    lens = [5, 13, 1, 9, 20]
+    T = sum(lens)
+    rng = np.random.default_rng(12)
+    Qall = rng.standard_normal((T, Hq, d))
+    nKall = -(-T // B)
+    pages_k = rng.standard_normal((nKall + 2, Hkv, B, d))
+    pages_v = rng.standard_normal((nKall + 2, Hkv, B, d))
+    pt_all = rng.permutation(nKall + 2)[:nKall]
+    Kf = oracle.depage(pages_k, pt_all, nKall)[:, :T]
+    Vf = oracle.depage(pages_v, pt_all, nKall)[:, :T]
+    causal = np.arange(T)[None, :] <= np.arange(T)[:, None]
+    Oref, Lref = sdpa_reference(Qall, Kf, Vf, np.broadcast_to(causal, (Hq, T, T)).copy(), Hq // Hkv)
+    P = 0
+    for Lc in lens:
+        nQ, nK = -(-Lc // B), -(-(P + Lc) // B)
+        m = workloads.ones_mask(Hq, P // B, nQ, nK, workloads.last_live_block(P, Lc, B))
+        t, c = oracle.oracle_tables(m, Hkv)
+        O, L = oracle.oracle_chunk_attention(Qall[P:P + Lc], pages_k, pages_v, pt_all[:nK], t, c, P)
+        np.testing.assert_allclose(O, Oref[P:P + Lc], atol=1e-10)
+        np.testing.assert_allclose(L, Lref[:, P:P + Lc], atol=1e-10)
+        P += Lc
+
+
+def test_varlen_equals_independent_sequences():
+    """A batch over one page pool = each sequence on its own (SDPA per sequence)."""
+    Hq, Hkv, d, B = 4, 2, 8, 8
+    seqs = [(19, 6), (0, 17), (40, 1), (8, 8)]          # (prefix, chunk)
+    rng = np.random.default_rng(5)
+    nKs = [-(-(P + L) // B) for P, L in seqs]
+    num_pages = sum(nKs) + 3
+    perm = rng.permutation(num_pages)
+    Kp = rng.standard_normal((num_pages, Hkv, B, d))
+    Vp = rng.standard_normal((num_pages, Hkv, B, d))
+    cu_q = np.concatenate([[0], np.cumsum([L for _, L in seqs])])
+    cu_pages = np.concatenate([[0], np.cumsum(nKs)])
+    Q = rng.standard_normal((cu_q[-1], Hq, d))
+    tables, counts = [], []
+    for s, (P, L) in enumerate(seqs):
+        m = workloads.bernoulli_mask(Hq, P // B, -(-L // B), nKs[s], 0.4, seed=s,
+                                     last=workloads.last_live_block(P, L, B))
+        t, c = oracle.oracle_tables(m, Hkv)
+        tables.append(t.reshape(-1))
+        counts.append(c)
+    O, LSE = oracle.oracle_varlen(Q, Kp, Vp, cu_q, [P for P, _ in seqs], perm[:cu_pages[-1]],
+                                  cu_pages, np.concatenate(tables), np.stack(counts))
+    for s, (P, L) in enumerate(seqs):
+        pt = perm[cu_pages[s]:cu_pages[s + 1]]
+        t = tables[s].reshape(Hkv, nKs[s])
+        Kf, Vf = oracle.depage(Kp, pt, nKs[s]), oracle.depage(Vp, pt, nKs[s])
+        vis = token_visibility(t, counts[s], Hq, Hkv, P, L, B, nKs[s])
+        Or, Lr = sdpa_reference(Q[cu_q[s]:cu_q[s + 1]], Kf, Vf, vis, Hq // Hkv)
+        np.testing.assert_allclose(O[cu_q[s]:cu_q[s + 1]], Or, atol=1e-10)
+        np.testing.assert_allclose(LSE[:, cu_q[s]:cu_q[s + 1]], Lr, atol=1e-10)

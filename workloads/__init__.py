@@ -14,4 +14,5 @@ from .generators import (  # noqa: F401
     pack_mask_bits,
     mask_for,
     causal_live,
+    last_live_block,
 )

@@ -34,12 +34,12 @@ class Workload:
         return self.prefix_len // self.block
 
     @property
-    def nQblk(self):
-        return self.chunk_len // self.block
+    def nQblk(self):  # Q-block qb = chunk tokens [qb B, qb B + B); the last may be partial
+        return -(-self.chunk_len // self.block)
 
     @property
-    def nKblk(self):
-        return (self.prefix_len + self.chunk_len) // self.block
+    def nKblk(self):  # KV block kb = positions [kb B, kb B + B); the last may be partial
+        return -(-(self.prefix_len + self.chunk_len) // self.block)
 
     @property
     def num_pages(self):

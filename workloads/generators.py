@@ -41,30 +41,43 @@ def make_qkv_pages(w, seed=None, num_pages=None, identity_pages=False):
     return {"Q": q, "K_pages": k, "V_pages": v, "page_table": torch.from_numpy(pt)}
 
 
-def causal_live(nPblk, nQblk, nKblk):
+def last_live_block(P, L, B):
+    """int [nQblk]: the last KV block holding a position visible to Q-block qb
+    (chunk tokens [qb B, min(qb B + B, L)) at positions P + t).  For block-aligned
+    P and L it is the diagonal block nPblk + qb."""
+    nQ = -(-L // B)
+    qb = np.arange(nQ)
+    return (P + np.minimum(qb * B + B - 1, L - 1)) // B
+
+
+def _last(nPblk, nQblk, last):
+    return nPblk + np.arange(nQblk) if last is None else np.asarray(last)
+
+
+def causal_live(nPblk, nQblk, nKblk, last=None):
     """bool [nQblk, nKblk]: KV block kb can hold a key visible to Q-block qb."""
-    qb = np.arange(nQblk)[:, None]
     kb = np.arange(nKblk)[None, :]
-    return kb <= nPblk + qb
+    return kb <= _last(nPblk, nQblk, last)[:, None]
 
 
-def _sink_diag(nPblk, nQblk, nKblk):
-    qb = np.arange(nQblk)[:, None]
+def _sink_diag(nPblk, nQblk, nKblk, last=None):
     kb = np.arange(nKblk)[None, :]
-    return (kb == 0) | (kb == nPblk + qb)
+    return (kb == 0) | (kb == _last(nPblk, nQblk, last)[:, None])
 
 
-def bernoulli_mask(Hq, nPblk, nQblk, nKblk, rho, seed, clip=True):
-    """i.i.d. Bernoulli(rho) blocks, plus the sink block and the diagonal block."""
+def bernoulli_mask(Hq, nPblk, nQblk, nKblk, rho, seed, clip=True, last=None):
+    """i.i.d. Bernoulli(rho) blocks, plus the sink block and the diagonal block
+    (the last live block of each Q-block)."""
     rng = np.random.default_rng(seed)
     m = rng.random((Hq, nQblk, nKblk)) < rho
-    m |= _sink_diag(nPblk, nQblk, nKblk)[None]
+    m |= _sink_diag(nPblk, nQblk, nKblk, last)[None]
     if clip:
-        m &= causal_live(nPblk, nQblk, nKblk)[None]
+        m &= causal_live(nPblk, nQblk, nKblk, last)[None]
     return m.astype(np.uint8)
 
 
-def vertical_slash_mask(Hq, Hkv, nPblk, nQblk, nKblk, rho_col, corr, window, seed, clip=True):
+def vertical_slash_mask(Hq, Hkv, nPblk, nQblk, nKblk, rho_col, corr, window, seed, clip=True,
+                        last=None):
     """Vertical columns shared within a GQA group with probability ``corr``,
     a sink block, and a local window of ``window`` blocks ending at the diagonal.
 
@@ -78,30 +91,31 @@ def vertical_slash_mask(Hq, Hkv, nPblk, nQblk, nKblk, rho_col, corr, window, see
     own = rng.random((Hq, nKblk)) < rho_col
     pick = rng.random((Hq, nKblk)) < corr
     cols = np.where(pick, np.repeat(shared, G, axis=0), own)
-    qb = np.arange(nQblk)[:, None]
     kb = np.arange(nKblk)[None, :]
-    slash = (kb == 0) | ((kb > nPblk + qb - window) & (kb <= nPblk + qb))
+    lastc = _last(nPblk, nQblk, last)[:, None]
+    slash = (kb == 0) | ((kb > lastc - window) & (kb <= lastc))
     m = cols[:, None, :] | slash[None]
     if clip:
-        m &= causal_live(nPblk, nQblk, nKblk)[None]
+        m &= causal_live(nPblk, nQblk, nKblk, last)[None]
     return m.astype(np.uint8)
 
 
-def ones_mask(Hq, nPblk, nQblk, nKblk):
+def ones_mask(Hq, nPblk, nQblk, nKblk, last=None):
     """Every causally live block selected (the density-100% case)."""
-    live = causal_live(nPblk, nQblk, nKblk)
+    live = causal_live(nPblk, nQblk, nKblk, last)
     return np.broadcast_to(live[None], (Hq, nQblk, nKblk)).astype(np.uint8).copy()
 
 
 def mask_for(w, seed=None, clip=True):
     seed = w.seed if seed is None else seed
+    last = last_live_block(w.prefix_len, w.chunk_len, w.block)
     if w.mask_kind == "bernoulli":
-        return bernoulli_mask(w.Hq, w.nPblk, w.nQblk, w.nKblk, w.rho, seed, clip)
+        return bernoulli_mask(w.Hq, w.nPblk, w.nQblk, w.nKblk, w.rho, seed, clip, last)
     if w.mask_kind == "vslash":
         return vertical_slash_mask(w.Hq, w.Hkv, w.nPblk, w.nQblk, w.nKblk, w.rho, w.corr,
-                                   w.window, seed, clip)
+                                   w.window, seed, clip, last)
     if w.mask_kind == "ones":
-        return ones_mask(w.Hq, w.nPblk, w.nQblk, w.nKblk)
+        return ones_mask(w.Hq, w.nPblk, w.nQblk, w.nKblk, last)
     raise ValueError(w.mask_kind)
 
 
