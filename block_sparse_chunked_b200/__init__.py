@@ -26,6 +26,8 @@ from ._capi import (  # noqa: F401
     build_tables_bits,
     workspace_size,
     chunk_attention,
+    chunk_attention_varlen,
+    chunk_attention_masked,
     append_kv,
     check,
     wait_probe,

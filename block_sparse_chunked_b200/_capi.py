@@ -34,6 +34,15 @@ EXPORTS = {
                                             _c_int, _c_int, _c_int, _c_int, _vp, _vp, _c_int,
                                             _vp, _vp]),
     "ca_noalloc_scratch_bytes": (_c_size, []),
+    "ca_workspace_size_varlen": (_c_size, [_c_int] * 10),
+    "ca_workspace_size_masked": (_c_size, [_c_int] * 9),
+    "ca_chunk_attention_masked": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _c_int, _c_int,
+                                           _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp,
+                                           _vp, _c_size, _c_int, _vp, _vp]),
+    "ca_chunk_attention_varlen": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp,
+                                           _vp, _c_int, _vp, _vp, _vp, _vp, _c_int, _c_int,
+                                           _c_int, _c_int, _vp, _vp, _vp, _c_size, _c_int, _vp,
+                                           _vp]),
     "ca_append_kv": (_c_int, [_vp, _vp, _c_int, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int,
                               _c_int, _c_int, _vp, _vp]),
     "ca_check": (_c_int, [_vp, _vp]),
@@ -172,7 +181,7 @@ def chunk_attention(Q, K_pages, V_pages, page_table, tables, counts, prefix_len,
     num_pages, Hkv, B, d2 = K_pages.shape
     if d2 != d:
         raise ValueError("head_dim of Q and of the pages differ")
-    nK = (prefix_len + L) // B if B else 0
+    nK = -(-(prefix_len + L) // B) if B else 0
     if page_table.numel() < nK or tables.shape[0] != Hkv or tables.shape[1] < nK \
             or counts.numel() < Hkv:
         raise ValueError("page_table / tables / counts are smaller than the chunk needs")
@@ -188,6 +197,90 @@ def chunk_attention(Q, K_pages, V_pages, page_table, tables, counts, prefix_len,
         _ptr(Q), _ptr(K_pages), _ptr(V_pages), code, num_pages, _ptr(page_table), _ptr(tables),
         _ptr(counts), Hq, Hkv, d, B, L, prefix_len, _ptr(out), _ptr(lse),
         _ptr(workspace) if ws_n else None, ws_n, n_splits, _ptr(err_flag), _stream()))
+    return out, lse
+
+
+def chunk_attention_masked(Q, K_pages, V_pages, page_table, mask_bits, prefix_len, n_splits=0,
+                           err_flag=None, out=None, lse=None, tables_out=None, counts_out=None,
+                           workspace=None):
+    """Attention with the table builder fused in: mask_bits int32/uint32
+    [Hq, nQblk, ceil(nKblk/32)] instead of tables.  Optionally writes the
+    tables to tables_out [Hkv, nKblk] / counts_out [Hkv].  Returns O and LSE."""
+    _need_cuda("Q", Q, tuple(_DT), 3)
+    _need_cuda("K_pages", K_pages, (Q.dtype,), 4)
+    _need_cuda("V_pages", V_pages, (Q.dtype,), 4)
+    _need_cuda("page_table", page_table, (torch.int32,), 1)
+    _need_cuda("mask_bits", mask_bits, (torch.int32, torch.uint32), 3)
+    if K_pages.shape != V_pages.shape:
+        raise ValueError("K_pages and V_pages must have the same shape")
+    L, Hq, d = Q.shape
+    num_pages, Hkv, B, d2 = K_pages.shape
+    nK = -(-(prefix_len + L) // B)
+    if d2 != d or tuple(mask_bits.shape) != (Hq, -(-L // B), (nK + 31) // 32) \
+            or page_table.numel() < nK:
+        raise ValueError("mask_bits / page_table do not match the chunk")
+    for name, t, n in (("tables_out", tables_out, Hkv * nK), ("counts_out", counts_out, Hkv)):
+        if t is not None:
+            _need_cuda(name, t, (torch.int32,))
+            if t.numel() < n:
+                raise ValueError(f"{name} is too small")
+    code = _DT[Q.dtype]
+    if out is None:
+        out = torch.empty_like(Q)
+    if lse is None:
+        lse = torch.empty(Hq, L, dtype=torch.float32, device=Q.device)
+    ws_n = lib.ca_workspace_size_masked(code, Hq, Hkv, d, B, L, prefix_len, num_pages, n_splits)
+    if ws_n == ctypes.c_size_t(-1).value:
+        raise CompactAttnError(CA_ERR_ARG, "invalid shapes for ca_workspace_size_masked")
+    if ws_n and (workspace is None or workspace.numel() < ws_n):
+        workspace = torch.empty(ws_n, dtype=torch.uint8, device=Q.device)
+    _ok(lib.ca_chunk_attention_masked(
+        _ptr(Q), _ptr(K_pages), _ptr(V_pages), code, num_pages, _ptr(page_table), _ptr(mask_bits),
+        Hq, Hkv, d, B, L, prefix_len, _ptr(tables_out), _ptr(counts_out), _ptr(out), _ptr(lse),
+        _ptr(workspace) if ws_n else None, ws_n, n_splits, _ptr(err_flag), _stream()))
+    return out, lse
+
+
+def chunk_attention_varlen(Q, K_pages, V_pages, cu_q, prefix_len, page_table, cu_pages, tables,
+                           counts, max_kv_len, n_splits=1, err_flag=None, out=None, lse=None,
+                           workspace=None):
+    """Chunk attention for a batch of sequences over one page pool.
+
+    Q [total_q, Hq, d]; cu_q int32 [S+1] (row offsets); prefix_len int32 [S];
+    page_table int32 (concatenated, sequence s from cu_pages[s]); cu_pages int32
+    [S+1]; tables int32 (flat: sequence s's [Hkv, nKblk_s] from Hkv*cu_pages[s]);
+    counts int32 [S, Hkv]; max_kv_len >= every P_s + L_s.  All on the device.
+    Returns O [total_q, Hq, d] and LSE float32 [Hq, total_q].
+    """
+    _need_cuda("Q", Q, tuple(_DT), 3)
+    _need_cuda("K_pages", K_pages, (Q.dtype,), 4)
+    _need_cuda("V_pages", V_pages, (Q.dtype,), 4)
+    for name, t in (("cu_q", cu_q), ("prefix_len", prefix_len), ("page_table", page_table),
+                    ("cu_pages", cu_pages), ("tables", tables), ("counts", counts)):
+        _need_cuda(name, t, (torch.int32,))
+    if K_pages.shape != V_pages.shape:
+        raise ValueError("K_pages and V_pages must have the same shape")
+    total_q, Hq, d = Q.shape
+    num_pages, Hkv, B, d2 = K_pages.shape
+    S = prefix_len.numel()
+    if d2 != d or cu_q.numel() != S + 1 or cu_pages.numel() != S + 1 or counts.numel() < S * Hkv:
+        raise ValueError("inconsistent batch arrays")
+    code = _DT[Q.dtype]
+    if out is None:
+        out = torch.empty_like(Q)
+    if lse is None:
+        lse = torch.empty(Hq, total_q, dtype=torch.float32, device=Q.device)
+    ws_n = lib.ca_workspace_size_varlen(code, Hq, Hkv, d, B, S, total_q, max_kv_len, num_pages,
+                                        n_splits)
+    if ws_n == ctypes.c_size_t(-1).value:
+        raise CompactAttnError(CA_ERR_ARG, "invalid shapes for ca_workspace_size_varlen")
+    if workspace is None or workspace.numel() < ws_n:
+        workspace = torch.empty(ws_n, dtype=torch.uint8, device=Q.device)
+    _ok(lib.ca_chunk_attention_varlen(
+        _ptr(Q), _ptr(K_pages), _ptr(V_pages), code, num_pages, S, total_q, _ptr(cu_q),
+        _ptr(prefix_len), max_kv_len, _ptr(page_table), _ptr(cu_pages), _ptr(tables),
+        _ptr(counts), Hq, Hkv, d, B, _ptr(out), _ptr(lse), _ptr(workspace), ws_n, n_splits,
+        _ptr(err_flag), _stream()))
     return out, lse
 
 

@@ -62,34 +62,35 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 constexpr int kMaxPersistentUnits = 2048;  // units whose schedule a CTA keeps in shared memory
 
 struct Plan {
-  int G, HPU, NT, nhalves, nqs, nPblk, nKblk, spb, n_splits;
+  int G, HPU, NT, nhalves, spb, n_splits;
   int units, persistent, sk_ctas;
 };
 
-bool plan(int Hq, int Hkv, int head_dim, int block, int chunk_len, int prefix_len, int n_splits,
-          Plan& pl) {
+// Heads -> tiles: a unit stacks up to four heads of a group over a 64-token
+// span (two heads per 128-row tile).
+bool plan_heads(int Hq, int Hkv, int head_dim, int block, Plan& pl) {
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return false;
   if (head_dim != 64 && head_dim != 128) return false;
   if (block != 64 && block != 128) return false;
-  if (chunk_len < 64 || prefix_len < 0) return false;
-  if (chunk_len % block || prefix_len % block) return false;
   pl.G = Hq / Hkv;
   pl.HPU = pl.G < 4 ? pl.G : 4;
   pl.NT = (pl.HPU + 1) / 2;
   pl.nhalves = (pl.G + pl.HPU - 1) / pl.HPU;
-  pl.nqs = chunk_len / 64;
-  pl.nPblk = prefix_len / block;
-  pl.nKblk = (prefix_len + chunk_len) / block;
   pl.spb = 128 / block;
-  const long long units = (long long)Hkv * pl.nhalves * pl.nqs;
-  const int max_stages = (pl.nKblk + pl.spb - 1) / pl.spb;
-  pl.units = (int)std::min<long long>(units, 0x7fffffff);
+  return true;
+}
+
+// Work mode for `units` units of at most `max_stages` KV stages each.
+bool plan_mode(Plan& pl, long long units, int max_stages, int n_splits, bool allow_persistent) {
+  if (units > 0x7fffffffLL) return false;
+  pl.units = (int)units;
   // Automatic mode: one CTA per unit when the units fill the SMs; otherwise a
   // persistent grid of at most one CTA per SM, each taking an equal share of
   // all units' KV stages (at least ~4 stages per CTA).  (At 256 units on 148
   // SMs the persistent grid measured 5% slower than one CTA per unit: the
   // piece boundaries and the merge cost more than the balance gains.)
-  pl.persistent = (n_splits <= 0 && units < kSMs && units <= kMaxPersistentUnits) ? 1 : 0;
+  pl.persistent = (allow_persistent && n_splits <= 0 && units < kSMs && units <= kMaxPersistentUnits)
+                      ? 1 : 0;
   if (n_splits <= 0 && !pl.persistent) n_splits = 1;
   pl.sk_ctas = 0;
   if (pl.persistent) {
@@ -99,11 +100,6 @@ bool plan(int Hq, int Hkv, int head_dim, int block, int chunk_len, int prefix_le
     return true;
   }
   int S = n_splits;
-  if (S <= 0) {
-    S = 1;
-    if (units < kSMs) S = (int)((2 * kSMs + units - 1) / units);
-    if (S > 16) S = 16;
-  }
   if (S > max_stages) S = max_stages;
   if (S < 1) S = 1;
   if (units * S > 0x7fffffffLL) return false;
@@ -111,35 +107,64 @@ bool plan(int Hq, int Hkv, int head_dim, int block, int chunk_len, int prefix_le
   return true;
 }
 
+// One sequence: chunk_len >= 1 tokens after prefix_len >= 0 tokens (no
+// alignment needed: masks hold Q-blocks of the chunk's tokens and KV blocks
+// of the sequence's positions).
+bool plan(int Hq, int Hkv, int head_dim, int block, int chunk_len, int prefix_len, int n_splits,
+          Plan& pl, SeqDesc& d) {
+  if (!plan_heads(Hq, Hkv, head_dim, block, pl)) return false;
+  if (chunk_len < 1 || prefix_len < 0 || (long long)prefix_len + chunk_len > 0x7fffffffLL)
+    return false;
+  d.q_start = 0;
+  d.L = chunk_len;
+  d.P = prefix_len;
+  d.nKblk = (int)(((long long)prefix_len + chunk_len + block - 1) / block);
+  d.pt_off = 0;
+  d.unit_start = 0;
+  d.nqs = (chunk_len + 63) / 64;
+  d.seq = 0;
+  const long long units = (long long)Hkv * pl.nhalves * d.nqs;
+  const int max_stages = (d.nKblk + pl.spb - 1) / pl.spb;
+  return plan_mode(pl, units, max_stages, n_splits, true);
+}
+
 struct WsLayout {
   size_t opart = 0, lsepart = 0, q = 0, qlo = 0, k = 0, v = 0, sched = 0, osk = 0, lsesk = 0,
-         total = 0;
+         seqs = 0, nunits = 0, total = 0;
 };
 
-WsLayout ws_layout(int dtype, int Hq, int Hkv, int D, int B, int L, int num_pages, const Plan& pl) {
+// rows = rows of Q / O; num_seqs > 0 reserves the batched call's descriptors.
+WsLayout ws_layout(int dtype, int Hq, int Hkv, int D, int B, long long rows, int num_pages,
+                   const Plan& pl, int num_seqs = 0) {
   WsLayout w;
   size_t off = 0;
   const int S = pl.n_splits;
+  if (num_seqs > 0) {
+    w.seqs = off;
+    off = align256(off + (size_t)num_seqs * sizeof(SeqDesc));
+    w.nunits = off;
+    off = align256(off + 4);
+  }
   if (pl.persistent) {
-    const size_t rows = (size_t)pl.NT * 128;
+    const size_t trows = (size_t)pl.NT * 128;
     w.sched = off;
     off = align256(off + (size_t)(pl.units + 1) * 4);
     w.osk = off;
-    off = align256(off + 2 * (size_t)pl.sk_ctas * rows * D * 4);
+    off = align256(off + 2 * (size_t)pl.sk_ctas * trows * D * 4);
     w.lsesk = off;
-    off = align256(off + 2 * (size_t)pl.sk_ctas * rows * 4);
+    off = align256(off + 2 * (size_t)pl.sk_ctas * trows * 4);
   }
   if (S > 1) {
     w.opart = off;
-    off = align256(off + (size_t)S * L * Hq * D * 4);
+    off = align256(off + (size_t)S * rows * Hq * D * 4);
     w.lsepart = off;
-    off = align256(off + (size_t)S * Hq * L * 4);
+    off = align256(off + (size_t)S * Hq * rows * 4);
   }
   if (dtype == CA_DTYPE_FP32) {
     w.q = off;
-    off = align256(off + (size_t)L * Hq * D * 2);
+    off = align256(off + (size_t)rows * Hq * D * 2);
     w.qlo = off;
-    off = align256(off + (size_t)L * Hq * D * 2);
+    off = align256(off + (size_t)rows * Hq * D * 2);
     w.k = off;
     off = align256(off + (size_t)num_pages * Hkv * B * D * 2);
     w.v = off;
@@ -147,6 +172,11 @@ WsLayout ws_layout(int dtype, int Hq, int Hkv, int D, int B, int L, int num_page
   }
   w.total = off;
   return w;
+}
+
+// Units bound of a batched call: sum_s ceil(L_s / 64) <= total_q / 64 + num_seqs.
+long long varlen_units_bound(int total_q, int num_seqs, int Hkv, int nhalves) {
+  return ((long long)(total_q + 63) / 64 + num_seqs) * Hkv * nhalves;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -214,47 +244,36 @@ int ca_build_tables_bits(const uint32_t* mask_bits, int nb, int Hq, int Hkv, int
 size_t ca_workspace_size(int dtype, int Hq, int Hkv, int head_dim, int block, int chunk_len,
                          int prefix_len, int num_pages, int n_splits) {
   Plan pl;
+  SeqDesc d;
   if (dtype != CA_DTYPE_BF16 && dtype != CA_DTYPE_FP32) return (size_t)-1;
-  if (!plan(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl)) return (size_t)-1;
-  if (num_pages < pl.nKblk) return (size_t)-1;
+  if (!plan(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl, d)) return (size_t)-1;
+  if (num_pages < d.nKblk) return (size_t)-1;
   return ws_layout(dtype, Hq, Hkv, head_dim, block, chunk_len, num_pages, pl).total;
 }
 
-int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, int dtype,
-                       int num_pages, const int32_t* page_table, const int32_t* tables,
-                       const int32_t* counts, int Hq, int Hkv, int head_dim, int block,
-                       int chunk_len, int prefix_len, void* O, float* LSE, void* workspace,
-                       size_t ws_bytes, int n_splits, int32_t* err_flag, void* stream) {
-  if (!Q || !K_pages || !V_pages || !page_table || !tables || !counts || !O || !LSE)
-    return fail(CA_ERR_ARG, "ca_chunk_attention: null pointer");
-  if (dtype != CA_DTYPE_BF16 && dtype != CA_DTYPE_FP32)
-    return fail(CA_ERR_DTYPE, "ca_chunk_attention: dtype code %d not supported", dtype);
-  if (block != 64 && block != 128)
-    return fail(CA_ERR_ARG, "ca_chunk_attention: block=%d must be 64 or 128", block);
-  if (chunk_len % block || prefix_len % block)
-    return fail(CA_ERR_ALIGN,
-                "ca_chunk_attention: prefix_len=%d and chunk_len=%d must be multiples of block=%d",
-                prefix_len, chunk_len, block);
+size_t ca_workspace_size_varlen(int dtype, int Hq, int Hkv, int head_dim, int block, int num_seqs,
+                                int total_q, int max_kv_len, int num_pages, int n_splits) {
   Plan pl;
-  if (!plan(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl))
-    return fail(CA_ERR_ARG,
-                "ca_chunk_attention: unsupported shape Hq=%d Hkv=%d head_dim=%d block=%d "
-                "chunk_len=%d prefix_len=%d",
-                Hq, Hkv, head_dim, block, chunk_len, prefix_len);
-  if (num_pages < pl.nKblk)
-    return fail(CA_ERR_ARG, "ca_chunk_attention: num_pages=%d < nKblk=%d", num_pages, pl.nKblk);
-  if (!aligned16(Q) || !aligned16(K_pages) || !aligned16(V_pages) || !aligned16(O))
-    return fail(CA_ERR_ARG, "ca_chunk_attention: Q, K_pages, V_pages and O must be 16-byte aligned");
-  const WsLayout wl = ws_layout(dtype, Hq, Hkv, head_dim, block, chunk_len, num_pages, pl);
-  if (wl.total > 0 && (!workspace || ws_bytes < wl.total || !aligned16(workspace)))
-    return fail(CA_ERR_WORKSPACE, "ca_chunk_attention: workspace of %zu bytes needed, got %zu",
-                wl.total, workspace ? ws_bytes : (size_t)0);
-  EncodeTiledFn enc = encoder();
-  if (!enc) return fail(CA_ERR_LAUNCH, "ca_chunk_attention: cuTensorMapEncodeTiled unavailable");
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const int D = head_dim, B = block, L = chunk_len;
+  if (dtype != CA_DTYPE_BF16 && dtype != CA_DTYPE_FP32) return (size_t)-1;
+  if (num_seqs < 1 || total_q < 0 || max_kv_len < 0 || num_pages < 1) return (size_t)-1;
+  if (!plan_heads(Hq, Hkv, head_dim, block, pl)) return (size_t)-1;
+  const int max_stages = std::max(1, (max_kv_len + 127) / 128);
+  if (!plan_mode(pl, varlen_units_bound(total_q, num_seqs, Hkv, pl.nhalves), max_stages,
+                 n_splits, false))
+    return (size_t)-1;
+  return ws_layout(dtype, Hq, Hkv, head_dim, block, total_q, num_pages, pl, num_seqs).total;
+}
 
+namespace {
+
+// Shared tail of the attention entry points: fp32 casts, tensor maps, launch,
+// merges.  `p` arrives with the sequence fields set; rows = rows of Q / O.
+int run_attention(const char* who, const void* Q, const void* K_pages, const void* V_pages,
+                  int dtype, int num_pages, int Hq, int Hkv, int D, int B, int rows,
+                  const Plan& pl, const WsLayout& wl, uint8_t* ws, int grid, AttnParams& p,
+                  cudaStream_t st) {
+  EncodeTiledFn enc = encoder();
+  if (!enc) return fail(CA_ERR_LAUNCH, "%s: cuTensorMapEncodeTiled unavailable", who);
   const void* q = Q;
   const void* qlo = Q;
   const void* kp = K_pages;
@@ -265,14 +284,14 @@ int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, 
     // bf16 terms (its rounding error would shift every score of a row the
     // same way); K and V are rounded once.
     e = launch_split_f32_bf16(static_cast<const float*>(Q), ws + wl.q, ws + wl.qlo,
-                              (size_t)L * Hq * D, st);
+                              (size_t)rows * Hq * D, st);
     if (e == cudaSuccess)
       e = launch_cast_f32_bf16(static_cast<const float*>(K_pages), ws + wl.k,
                                (size_t)num_pages * Hkv * B * D, st);
     if (e == cudaSuccess)
       e = launch_cast_f32_bf16(static_cast<const float*>(V_pages), ws + wl.v,
                                (size_t)num_pages * Hkv * B * D, st);
-    if (e != cudaSuccess) return cuda_fail(e, "ca_chunk_attention cast");
+    if (e != cudaSuccess) return cuda_fail(e, "cast to bf16");
     q = ws + wl.q;
     qlo = ws + wl.qlo;
     kp = ws + wl.k;
@@ -281,7 +300,8 @@ int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, 
 
   CUtensorMap tq, tqlo, tk, tv;
   for (int which = 0; which < 2; ++which) {
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)L};
+    // rows beyond the last are zero-filled by the copy engine (a ragged last span)
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)std::max(rows, 1)};
     cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
     cuuint32_t box[3] = {64, 1, 64};
     cuuint32_t es[3] = {1, 1, 1};
@@ -289,7 +309,7 @@ int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, 
                      const_cast<void*>(which ? qlo : q), dims, strides, box, es,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(CA_ERR_LAUNCH, "tensor map (Q) encode failed: %d", (int)r);
+    if (r != CUDA_SUCCESS) return fail(CA_ERR_LAUNCH, "%s: tensor map (Q) encode failed: %d", who, (int)r);
   }
   for (int which = 0; which < 2; ++which) {
     cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)B, (cuuint64_t)Hkv, (cuuint64_t)num_pages};
@@ -302,19 +322,12 @@ int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, 
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
-      return fail(CA_ERR_LAUNCH, "tensor map (%s pages) encode failed: %d", which ? "V" : "K",
-                  (int)r);
+      return fail(CA_ERR_LAUNCH, "%s: tensor map (%s pages) encode failed: %d", who,
+                  which ? "V" : "K", (int)r);
   }
 
-  AttnParams p;
-  p.page_table = page_table;
-  p.tables = tables;
-  p.counts = counts;
-  p.O = O;
-  p.LSE = LSE;
   p.Opart = pl.n_splits > 1 ? reinterpret_cast<float*>(ws + wl.opart) : nullptr;
   p.LSEpart = pl.n_splits > 1 ? reinterpret_cast<float*>(ws + wl.lsepart) : nullptr;
-  p.err = err_flag;
   p.persistent = pl.persistent;
   p.n_units = pl.units;
   p.sk_ctas = pl.sk_ctas;
@@ -326,29 +339,194 @@ int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, 
   p.G = pl.G;
   p.HPU = pl.HPU;
   p.nhalves = pl.nhalves;
-  p.L = L;
-  p.P = prefix_len;
+  p.L = rows;
   p.B = B;
-  p.nPblk = pl.nPblk;
-  p.nKblk = pl.nKblk;
   p.num_pages = num_pages;
   p.n_splits = pl.n_splits;
-  p.nqs = pl.nqs;
   p.out_f32 = dtype == CA_DTYPE_FP32 ? 1 : 0;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   p.wait_ns = kWaitNs;
-  const int grid = pl.persistent ? pl.sk_ctas : Hkv * pl.nhalves * pl.nqs * pl.n_splits;
   e = launch_chunk_attention(tq, tqlo, tk, tv, p, D, pl.NT, dtype == CA_DTYPE_FP32, grid, st);
-  if (e != cudaSuccess) return cuda_fail(e, "ca_chunk_attention launch");
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   if (pl.persistent) {
     e = launch_sk_combine(p, D, pl.NT, st);
-    if (e != cudaSuccess) return cuda_fail(e, "ca_chunk_attention combine launch");
+    if (e != cudaSuccess) return cuda_fail(e, "attention combine launch");
   }
   if (pl.n_splits > 1) {
-    e = launch_split_combine(p.Opart, p.LSEpart, pl.n_splits, L, Hq, D, O, LSE, p.out_f32, st);
-    if (e != cudaSuccess) return cuda_fail(e, "ca_chunk_attention combine launch");
+    e = launch_split_combine(p.Opart, p.LSEpart, pl.n_splits, rows, Hq, D, p.O, p.LSE, p.out_f32, st);
+    if (e != cudaSuccess) return cuda_fail(e, "attention combine launch");
   }
   return CA_OK;
+}
+
+}  // namespace
+
+int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, int dtype,
+                       int num_pages, const int32_t* page_table, const int32_t* tables,
+                       const int32_t* counts, int Hq, int Hkv, int head_dim, int block,
+                       int chunk_len, int prefix_len, void* O, float* LSE, void* workspace,
+                       size_t ws_bytes, int n_splits, int32_t* err_flag, void* stream) {
+  if (!Q || !K_pages || !V_pages || !page_table || !tables || !counts || !O || !LSE)
+    return fail(CA_ERR_ARG, "ca_chunk_attention: null pointer");
+  if (dtype != CA_DTYPE_BF16 && dtype != CA_DTYPE_FP32)
+    return fail(CA_ERR_DTYPE, "ca_chunk_attention: dtype code %d not supported", dtype);
+  if (block != 64 && block != 128)
+    return fail(CA_ERR_ARG, "ca_chunk_attention: block=%d must be 64 or 128", block);
+  Plan pl;
+  SeqDesc d;
+  if (!plan(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl, d))
+    return fail(CA_ERR_ARG,
+                "ca_chunk_attention: unsupported shape Hq=%d Hkv=%d head_dim=%d block=%d "
+                "chunk_len=%d prefix_len=%d",
+                Hq, Hkv, head_dim, block, chunk_len, prefix_len);
+  if (num_pages < d.nKblk)
+    return fail(CA_ERR_ARG, "ca_chunk_attention: num_pages=%d < nKblk=%d", num_pages, d.nKblk);
+  if (!aligned16(Q) || !aligned16(K_pages) || !aligned16(V_pages) || !aligned16(O))
+    return fail(CA_ERR_ARG, "ca_chunk_attention: Q, K_pages, V_pages and O must be 16-byte aligned");
+  const WsLayout wl = ws_layout(dtype, Hq, Hkv, head_dim, block, chunk_len, num_pages, pl);
+  if (wl.total > 0 && (!workspace || ws_bytes < wl.total || !aligned16(workspace)))
+    return fail(CA_ERR_WORKSPACE, "ca_chunk_attention: workspace of %zu bytes needed, got %zu",
+                wl.total, workspace ? ws_bytes : (size_t)0);
+  AttnParams p{};
+  p.page_table = page_table;
+  p.tables = tables;
+  p.counts = counts;
+  p.O = O;
+  p.LSE = LSE;
+  p.err = err_flag;
+  p.n_units_dev = nullptr;
+  p.seqs = nullptr;
+  p.seq0 = d;
+  p.num_seqs = 1;
+  const int grid = pl.persistent ? pl.sk_ctas : pl.units * pl.n_splits;
+  return run_attention("ca_chunk_attention", Q, K_pages, V_pages, dtype, num_pages, Hq, Hkv,
+                       head_dim, block, chunk_len, pl, wl, static_cast<uint8_t*>(workspace), grid,
+                       p, static_cast<cudaStream_t>(stream));
+}
+
+namespace {
+// Fused calls: one CTA per unit (the table is built per CTA), KV splits when
+// the units do not fill the SMs.
+bool plan_masked(int Hq, int Hkv, int head_dim, int block, int chunk_len, int prefix_len,
+                 int n_splits, Plan& pl, SeqDesc& d) {
+  if (!plan(Hq, Hkv, head_dim, block, chunk_len, prefix_len, 1, pl, d)) return false;
+  if (d.nKblk > 2048) return false;
+  const int max_stages = (d.nKblk + pl.spb - 1) / pl.spb;
+  int S = n_splits;
+  if (S <= 0) S = pl.units >= kSMs ? 1 : (2 * kSMs + pl.units - 1) / pl.units;
+  if (S > 16 && n_splits <= 0) S = 16;
+  return plan_mode(pl, pl.units, max_stages, S, false);
+}
+}  // namespace
+
+size_t ca_workspace_size_masked(int dtype, int Hq, int Hkv, int head_dim, int block,
+                                int chunk_len, int prefix_len, int num_pages, int n_splits) {
+  Plan pl;
+  SeqDesc d;
+  if (dtype != CA_DTYPE_BF16 && dtype != CA_DTYPE_FP32) return (size_t)-1;
+  if (!plan_masked(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl, d))
+    return (size_t)-1;
+  if (num_pages < d.nKblk) return (size_t)-1;
+  return ws_layout(dtype, Hq, Hkv, head_dim, block, chunk_len, num_pages, pl).total;
+}
+
+int ca_chunk_attention_masked(const void* Q, const void* K_pages, const void* V_pages, int dtype,
+                              int num_pages, const int32_t* page_table, const uint32_t* mask_bits,
+                              int Hq, int Hkv, int head_dim, int block, int chunk_len,
+                              int prefix_len, int32_t* tables_out, int32_t* counts_out, void* O,
+                              float* LSE, void* workspace, size_t ws_bytes, int n_splits,
+                              int32_t* err_flag, void* stream) {
+  const char* who = "ca_chunk_attention_masked";
+  if (!Q || !K_pages || !V_pages || !page_table || !mask_bits || !O || !LSE)
+    return fail(CA_ERR_ARG, "%s: null pointer", who);
+  if (dtype != CA_DTYPE_BF16 && dtype != CA_DTYPE_FP32)
+    return fail(CA_ERR_DTYPE, "%s: dtype code %d not supported", who, dtype);
+  Plan pl;
+  SeqDesc d;
+  if (!plan_masked(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl, d))
+    return fail(CA_ERR_ARG,
+                "%s: unsupported shape Hq=%d Hkv=%d head_dim=%d block=%d chunk_len=%d "
+                "prefix_len=%d (nKblk <= 2048)",
+                who, Hq, Hkv, head_dim, block, chunk_len, prefix_len);
+  if (num_pages < d.nKblk)
+    return fail(CA_ERR_ARG, "%s: num_pages=%d < nKblk=%d", who, num_pages, d.nKblk);
+  if (!aligned16(Q) || !aligned16(K_pages) || !aligned16(V_pages) || !aligned16(O))
+    return fail(CA_ERR_ARG, "%s: Q, K_pages, V_pages and O must be 16-byte aligned", who);
+  if (reinterpret_cast<uintptr_t>(mask_bits) & 3u)
+    return fail(CA_ERR_ARG, "%s: mask_bits must be 4-byte aligned", who);
+  const WsLayout wl = ws_layout(dtype, Hq, Hkv, head_dim, block, chunk_len, num_pages, pl);
+  if (wl.total > 0 && (!workspace || ws_bytes < wl.total || !aligned16(workspace)))
+    return fail(CA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, got %zu", who, wl.total,
+                workspace ? ws_bytes : (size_t)0);
+  AttnParams p{};
+  p.page_table = page_table;
+  p.O = O;
+  p.LSE = LSE;
+  p.err = err_flag;
+  p.mask_bits = mask_bits;
+  p.mask_words = (d.nKblk + 31) / 32;
+  p.nQblk_mask = (chunk_len + block - 1) / block;
+  p.tables_out = tables_out;
+  p.counts_out = counts_out;
+  p.seq0 = d;
+  p.num_seqs = 1;
+  return run_attention(who, Q, K_pages, V_pages, dtype, num_pages, Hq, Hkv, head_dim, block,
+                       chunk_len, pl, wl, static_cast<uint8_t*>(workspace),
+                       pl.units * pl.n_splits, p, static_cast<cudaStream_t>(stream));
+}
+
+int ca_chunk_attention_varlen(const void* Q, const void* K_pages, const void* V_pages, int dtype,
+                              int num_pages, int num_seqs, int total_q, const int32_t* cu_q,
+                              const int32_t* prefix_len, int max_kv_len,
+                              const int32_t* page_table, const int32_t* cu_pages,
+                              const int32_t* tables, const int32_t* counts, int Hq, int Hkv,
+                              int head_dim, int block, void* O, float* LSE, void* workspace,
+                              size_t ws_bytes, int n_splits, int32_t* err_flag, void* stream) {
+  const char* who = "ca_chunk_attention_varlen";
+  if (!Q || !K_pages || !V_pages || !cu_q || !prefix_len || !page_table || !cu_pages ||
+      !tables || !counts || !O || !LSE)
+    return fail(CA_ERR_ARG, "%s: null pointer", who);
+  if (dtype != CA_DTYPE_BF16 && dtype != CA_DTYPE_FP32)
+    return fail(CA_ERR_DTYPE, "%s: dtype code %d not supported", who, dtype);
+  if (num_seqs < 1 || total_q < 0 || max_kv_len < 0 || num_pages < 1)
+    return fail(CA_ERR_ARG, "%s: num_seqs=%d total_q=%d max_kv_len=%d num_pages=%d", who,
+                num_seqs, total_q, max_kv_len, num_pages);
+  Plan pl;
+  if (!plan_heads(Hq, Hkv, head_dim, block, pl))
+    return fail(CA_ERR_ARG, "%s: unsupported shape Hq=%d Hkv=%d head_dim=%d block=%d", who, Hq,
+                Hkv, head_dim, block);
+  const int max_stages = std::max(1, (max_kv_len + 127) / 128);
+  if (!plan_mode(pl, varlen_units_bound(total_q, num_seqs, Hkv, pl.nhalves), max_stages,
+                 n_splits, false))
+    return fail(CA_ERR_ARG, "%s: too many work units", who);
+  if (!aligned16(Q) || !aligned16(K_pages) || !aligned16(V_pages) || !aligned16(O))
+    return fail(CA_ERR_ARG, "%s: Q, K_pages, V_pages and O must be 16-byte aligned", who);
+  const WsLayout wl = ws_layout(dtype, Hq, Hkv, head_dim, block, total_q, num_pages, pl, num_seqs);
+  if (!workspace || ws_bytes < wl.total || !aligned16(workspace))
+    return fail(CA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, got %zu", who, wl.total,
+                workspace ? ws_bytes : (size_t)0);
+  if (total_q == 0) return CA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  SeqDesc* seqs = reinterpret_cast<SeqDesc*>(ws + wl.seqs);
+  int32_t* n_units = reinterpret_cast<int32_t*>(ws + wl.nunits);
+  cudaError_t e = launch_varlen_setup(cu_q, prefix_len, cu_pages, num_seqs, total_q, block, Hkv,
+                                      pl.nhalves, seqs, n_units, err_flag, st);
+  if (e != cudaSuccess) return cuda_fail(e, "ca_chunk_attention_varlen setup launch");
+  AttnParams p{};
+  p.page_table = page_table;
+  p.tables = tables;
+  p.counts = counts;
+  p.O = O;
+  p.LSE = LSE;
+  p.err = err_flag;
+  p.n_units_dev = n_units;
+  p.seqs = seqs;
+  p.seq0 = SeqDesc{};
+  p.num_seqs = num_seqs;
+  const int grid = pl.units * pl.n_splits;
+  return run_attention(who, Q, K_pages, V_pages, dtype, num_pages, Hq, Hkv, head_dim, block,
+                       total_q, pl, wl, ws, grid, p, st);
 }
 
 int ca_check(int32_t* err_flag, void* stream) {

@@ -93,38 +93,127 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, const A
 // Number of work units whose stage counts a persistent CTA keeps in shared memory.
 constexpr int kMaxUnits = 2048;
 
-// Unit u -> (group, 64-token query span, head slice); later query spans
-// (more causal blocks) first.
+// The sequence that owns unit u.
+__device__ __forceinline__ SeqDesc seq_of(const AttnParams& p, int u) {
+  if (p.seqs == nullptr) return p.seq0;
+  int lo = 0, hi = p.num_seqs - 1;  // last sequence with unit_start <= u
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.seqs[mid].unit_start <= u) lo = mid;
+    else hi = mid - 1;
+  }
+  return p.seqs[lo];
+}
+
+// Unit u -> (sequence, group, 64-token query span, head slice); within a
+// sequence, later query spans (more causal blocks) first.
 struct UnitCoord {
+  SeqDesc d;
   int g, qs, hh;
 };
 __device__ __forceinline__ UnitCoord unit_coord(const AttnParams& p, int u) {
-  const int per_qs = p.Hkv * p.nhalves;
   UnitCoord c;
-  c.qs = p.nqs - 1 - u / per_qs;
-  c.g = (u % per_qs) / p.nhalves;
-  c.hh = (u % per_qs) % p.nhalves;
+  c.d = seq_of(p, u);
+  const int loc = u - c.d.unit_start;
+  const int per_qs = p.Hkv * p.nhalves;
+  c.qs = c.d.nqs - 1 - loc / per_qs;
+  c.g = (loc % per_qs) / p.nhalves;
+  c.hh = (loc % per_qs) % p.nhalves;
   return c;
 }
 
-// Live table entries of unit u: the entries <= its diagonal block, a prefix
-// of the ascending row (binary search).
+__device__ __forceinline__ const int32_t* table_row(const AttnParams& p, const UnitCoord& c) {
+  return p.tables + (size_t)c.d.pt_off * p.Hkv + (size_t)c.g * c.d.nKblk;
+}
+
+// Live table entries of unit u: the entries whose block can hold a key visible
+// to the span's last query (kb * B <= P + last token), a prefix of the
+// ascending row (binary search).
 __device__ __forceinline__ int unit_live(const AttnParams& p, int u) {
   const UnitCoord c = unit_coord(p, u);
-  const int diag_kb = p.nPblk + (c.qs * 64) / p.B;
-  const int32_t* trow = p.tables + (size_t)c.g * p.nKblk;
-  int cnt = p.counts[c.g];
-  if (cnt < 0 || cnt > p.nKblk) {
+  const int t_last = min(c.qs * 64 + 63, c.d.L - 1);
+  const int last_kb = (c.d.P + t_last) / p.B;
+  const int32_t* trow = table_row(p, c);
+  int cnt = p.counts[(size_t)c.d.seq * p.Hkv + c.g];
+  if (cnt < 0 || cnt > c.d.nKblk) {
     set_flag(p.err, CA_FLAG_BOUNDS);
-    cnt = cnt < 0 ? 0 : p.nKblk;
+    cnt = cnt < 0 ? 0 : c.d.nKblk;
   }
   int lo = 0, hi = cnt;
   while (lo < hi) {
     const int mid = (lo + hi) >> 1;
-    if (trow[mid] <= diag_kb) lo = mid + 1;
+    if (trow[mid] <= last_kb) lo = mid + 1;
     else hi = mid;
   }
   return lo;
+}
+
+// Fused mode: the unit's group table, built by the whole CTA from the
+// bit-packed masks (the Q-block union and intra-group union of the abstract,
+// then the compaction) into shared memory: fent[0 .. count) ascending,
+// followed (at fent + 2048) by the group's union bit set (mask_words words)
+// and the count.  Returns the count.
+constexpr int kMaxFusedWords = 64;  // nKblk <= 2048
+__device__ int fused_group_table(const AttnParams& p, const UnitCoord& uc, int32_t* fent,
+                                 int nthreads) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int W = p.mask_words;
+  uint32_t* uni = reinterpret_cast<uint32_t*>(fent + kMaxFusedWords * 32);
+  for (int w = tid; w < W; w += nthreads) uni[w] = 0u;
+  __syncthreads();
+  // OR down the group's G * nQblk rows: thread -> (vector v of a row, rows r,
+  // r + RT, ...), 16-byte loads when the rows allow, several loads in flight
+  const int R = p.G * p.nQblk_mask;
+  const uint32_t* base = p.mask_bits + (size_t)uc.g * R * W;
+  const bool vec4 = (W % 4) == 0 && (reinterpret_cast<uintptr_t>(p.mask_bits) & 15u) == 0;
+  const int NV = vec4 ? W / 4 : W;
+  const int RT = nthreads / NV;
+  if (tid < RT * NV) {
+    const int v = tid % NV;
+    if (vec4) {
+      uint4 acc = make_uint4(0u, 0u, 0u, 0u);
+      const uint4* rowp = reinterpret_cast<const uint4*>(base) + v;
+#pragma unroll 8
+      for (int r = tid / NV; r < R; r += RT) {
+        const uint4 x = __ldg(rowp + (size_t)r * NV);
+        acc.x |= x.x;
+        acc.y |= x.y;
+        acc.z |= x.z;
+        acc.w |= x.w;
+      }
+      if (acc.x) atomicOr(&uni[4 * v], acc.x);
+      if (acc.y) atomicOr(&uni[4 * v + 1], acc.y);
+      if (acc.z) atomicOr(&uni[4 * v + 2], acc.z);
+      if (acc.w) atomicOr(&uni[4 * v + 3], acc.w);
+    } else {
+      uint32_t acc = 0u;
+#pragma unroll 8
+      for (int r = tid / NV; r < R; r += RT) acc |= __ldg(base + (size_t)r * W + v);
+      if (acc) atomicOr(&uni[v], acc);
+    }
+  }
+  __syncthreads();
+  if (tid == 0 && (uc.d.nKblk & 31)) uni[W - 1] &= (1u << (uc.d.nKblk & 31)) - 1u;
+  __syncthreads();
+  // compaction by warp 0: lane l ranks words 2l and 2l + 1
+  int* total = reinterpret_cast<int*>(uni + kMaxFusedWords);
+  if (warp == 0) {
+    const int w0 = 2 * lane;
+    const uint32_t x0 = w0 < W ? uni[w0] : 0u, x1 = w0 + 1 < W ? uni[w0 + 1] : 0u;
+    const int cnt = __popc(x0) + __popc(x1);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int pos = incl - cnt;
+    for (uint32_t x = x0; x; x &= x - 1) fent[pos++] = w0 * 32 + __ffs(x) - 1;
+    for (uint32_t x = x1; x; x &= x - 1) fent[pos++] = (w0 + 1) * 32 + __ffs(x) - 1;
+    if (lane == 31) *total = incl;
+  }
+  __syncthreads();
+  return *total;
 }
 
 // How a piece's result leaves the CTA.
@@ -156,11 +245,15 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
   const uint32_t q_free = bars + 8u * (7 + 4 * kNS);
   int* misc = reinterpret_cast<int*>(sm + S::kMiscOff);
   // misc[0] tmem base, [1] live entries (one-piece mode), [2] first stage,
-  // [3] last stage (exclusive), [5] abort
+  // [3] last stage (exclusive), [4] live entries of the fused table (thread 0
+  // only), [5] abort
   volatile int* abort_flag = misc + 5;
   int* sk_live = reinterpret_cast<int*>(sm + S::kSchedOff);  // [kMaxUnits] (persistent)
   int* sk_pref = sk_live + kMaxUnits;                         // [kMaxUnits + 1]
 
+  // A batched call's grid is an upper bound on its units: surplus CTAs leave
+  // before touching shared memory, barriers or TMEM.
+  if (p.n_units_dev && !p.persistent && (int)(blockIdx.x / p.n_splits) >= *p.n_units_dev) return;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int spb = kStageKeys / p.B;  // pages per stage
@@ -169,10 +262,33 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
   // ---- work: one piece (one-piece mode) or a contiguous range of all
   // units' stages (persistent mode)
   if (threadIdx.x == 0) misc[5] = 0;
+  // fused mode keeps the group table here (the persistent schedule is not used then)
+  int32_t* fent = sk_live;
   if (!p.persistent) {
+    if (p.mask_bits) {
+      const int u = blockIdx.x / p.n_splits;
+      const UnitCoord uc = unit_coord(p, u);
+      const int cnt = fused_group_table(p, uc, fent, nthreads);
+      if (p.tables_out && uc.qs == 0 && uc.hh == 0 && blockIdx.x % p.n_splits == 0) {
+        int32_t* trow_out = p.tables_out + (size_t)uc.g * uc.d.nKblk;
+        for (int e = threadIdx.x; e < uc.d.nKblk; e += nthreads) trow_out[e] = e < cnt ? fent[e] : -1;
+        if (threadIdx.x == 0 && p.counts_out) p.counts_out[uc.g] = cnt;
+      }
+      if (threadIdx.x == 0) {
+        const int t_last = min(uc.qs * 64 + 63, uc.d.L - 1);
+        const int last_kb = (uc.d.P + t_last) / p.B;
+        int lo = 0, hi = cnt;
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (fent[mid] <= last_kb) lo = mid + 1;
+          else hi = mid;
+        }
+        misc[4] = lo;
+      }
+    }
     if (threadIdx.x == 0) {
       const int u = blockIdx.x / p.n_splits, split = blockIdx.x % p.n_splits;
-      const int live = unit_live(p, u);
+      const int live = p.mask_bits ? misc[4] : unit_live(p, u);
       const int nst = (live + spb - 1) / spb;
       misc[1] = live;
       misc[2] = (int)((long long)split * nst / p.n_splits);
@@ -284,7 +400,7 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
     for_each_piece([&](int u, int live, int s0, int s1, int, int) {
       if (s1 <= s0 || !ok) return;
       const UnitCoord uc = unit_coord(p, u);
-      const int32_t* trow = p.tables + (size_t)uc.g * p.nKblk;
+      const int32_t* trow = p.mask_bits ? fent : table_row(p, uc);
       if (pn > 0) ok = wait_warp(q_free, (pn - 1) & 1, p, abort_flag);
       if (ok && lane == 0) {
         mbar_expect_tx(q_full, S::kQTerms * NT * 128 * D * 2);
@@ -298,7 +414,7 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
               for (int c = 0; c < KCH; ++c)
                 tma_load_3d(sbase + S::kQOff + (q * NT + t) * S::kQTile + c * S::kChunkBytes +
                                 s * 64 * 128,
-                            q ? &tmQlo : &tmQ, q_full, c * 64, head, uc.qs * 64);
+                            q ? &tmQlo : &tmQ, q_full, c * 64, head, uc.d.q_start + uc.qs * 64);
             }
       }
       const int e_begin = s0 * spb, e_end = min(live, s1 * spb);
@@ -316,11 +432,11 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
             int pg = 0;
             if (my < e_end && my >= e_begin) {
               int kb = trow[my];
-              if (kb < 0 || kb >= p.nKblk) {
+              if (kb < 0 || kb >= uc.d.nKblk) {
                 set_flag(p.err, CA_FLAG_BOUNDS);
                 kb = 0;
               }
-              pg = p.page_table[kb];
+              pg = p.page_table[uc.d.pt_off + kb];
               if (pg < 0 || pg >= p.num_pages) {
                 set_flag(p.err, CA_FLAG_BOUNDS);
                 pg = 0;
@@ -471,23 +587,30 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
     for_each_piece([&](int u, int live, int s0, int s1, int out, int slot) {
       const UnitCoord uc = unit_coord(p, u);
       const int t0 = uc.qs * 64;
-      const int diag_kb = p.nPblk + t0 / p.B;
-      const int tok = t0 + (row & 63);
+      const int tl = t0 + (row & 63);     // token within the chunk
+      const int tok = uc.d.q_start + tl;  // row of Q / O
       const int hl_raw = uc.hh * p.HPU + 2 * t + sub;
-      const bool valid_row = (2 * t + sub) < p.HPU && hl_raw < p.G;
+      const bool valid_row = (2 * t + sub) < p.HPU && hl_raw < p.G && tl < uc.d.L;
       const int head = uc.g * p.G + min(hl_raw, p.G - 1);
-      const int nst = (live + spb - 1) / spb;
-      const int32_t* trow = p.tables + (size_t)uc.g * p.nKblk;
-      const bool has_diag = live > 0 && trow[live - 1] == diag_kb;
-      const int diag_lim = (t0 % p.B) + (row & 63);  // visible keys of the diagonal block: jl <= this
+      const int32_t* trow = p.mask_bits ? fent : table_row(p, uc);
+      // Token-level causal mask: only blocks that hold a key later than the
+      // span's first query (kb >= (P + t0) / B) need it; in the ascending
+      // table they are the last live entries, from mask_e on.
+      const int kb_m0 = (uc.d.P + t0) / p.B;
+      int mask_e = live;
+      while (mask_e > 0 && trow[mask_e - 1] >= kb_m0) --mask_e;
+      // those are consecutive blocks (at most the two the span's positions fall
+      // in): their first key positions
+      const int kposA = mask_e < live ? trow[mask_e] * p.B : 0;
+      const int kposB = kposA + p.B;
+      const int qpos = uc.d.P + tl;  // this row's position: keys j <= qpos are visible
       const int n = s1 - s0;
       float m_used = -INFINITY, l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
       for (int j = 0; j < n && ok; ++j) {
         const int stage = s0 + j, G = gj + j;
         const int npg = min(spb, live - stage * spb);
         const int nvalid = npg * p.B;
-        const bool diag_stage = has_diag && (stage == nst - 1);
-        const int diag_c0 = (npg - 1) * p.B;  // first column of the diagonal page
+        const bool mask_stage = stage * spb + npg > mask_e;
         ok = wait_warp(s_full(t), G & 1, p, abort_flag);
         if (!ok) break;
         tc_fence_after();
@@ -500,10 +623,16 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
 #pragma unroll
           for (int c = 64; c < kStageKeys; ++c) sr[c] = -INFINITY;
         }
-        if (diag_stage) {  // token-level causal mask, diagonal block only
+        if (mask_stage) {  // keys after this row's position -> -inf
+          // From the stage's first page that needs the mask, page pm, the key of
+          // column c >= pm * B is (its block) * B + (c - pm * B).
+          const int e0 = stage * spb;
+          const int pm = max(0, mask_e - e0);
+          const int cm0 = pm * p.B;
+          const int lim = qpos - (e0 + pm > mask_e ? kposB : kposA);  // visible while c - cm0 <= lim
 #pragma unroll
           for (int c = 0; c < kStageKeys; ++c)
-            if (c >= diag_c0 && (c - diag_c0) > diag_lim) sr[c] = -INFINITY;
+            if (c >= cm0 && (c - cm0) > lim) sr[c] = -INFINITY;
         }
         // row max of the raw scores (scale > 0 commutes with max)
         float mx0 = max3(sr[0], sr[1], sr[2]);
@@ -645,9 +774,10 @@ __global__ void __launch_bounds__(256)
   const int r = blockIdx.y * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   const UnitCoord uc = unit_coord(p, u);
   const int t = r >> 7, sub = (r >> 6) & 1;
-  const int tok = uc.qs * 64 + (r & 63);
+  const int tl = uc.qs * 64 + (r & 63);
+  const int tok = uc.d.q_start + tl;
   const int hl_raw = uc.hh * p.HPU + 2 * t + sub;
-  if (!((2 * t + sub) < p.HPU && hl_raw < p.G)) return;
+  if (!((2 * t + sub) < p.HPU && hl_raw < p.G && tl < uc.d.L)) return;
   const int head = uc.g * p.G + hl_raw;
   auto slot_of = [&](int c) { return (c == ca && cta_start(c) < a) ? 2 * c + 1 : 2 * c; };
   float m = -INFINITY;
@@ -753,6 +883,66 @@ __global__ void split_f32_bf16_kernel(const float* __restrict__ src, __nv_bfloat
   }
 }
 
+// Batched calls: per-sequence descriptors and unit offsets from the caller's
+// device arrays (one CTA, block-wide scan in chunks of blockDim.x sequences).
+// A sequence whose offsets are inconsistent gets no work units and flags
+// CA_FLAG_BOUNDS.
+__global__ void __launch_bounds__(1024)
+    varlen_setup_kernel(const int32_t* __restrict__ cu_q, const int32_t* __restrict__ prefix_len,
+                        const int32_t* __restrict__ cu_pages, int num_seqs, int total_q, int B,
+                        int Hkv, int nhalves, SeqDesc* __restrict__ out, int32_t* n_units,
+                        int32_t* err) {
+  __shared__ int warp_sum[32];
+  __shared__ int carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < num_seqs; base += blockDim.x) {
+    const int s = base + tid;
+    SeqDesc d = {0, 0, 0, 0, 0, 0, 0, s};
+    int units = 0;
+    if (s < num_seqs) {
+      const int q0 = cu_q[s], q1 = cu_q[s + 1], P = prefix_len[s];
+      const int p0 = cu_pages[s], p1 = cu_pages[s + 1];
+      const long long L = (long long)q1 - q0;
+      const long long nK = (P + L + B - 1) / B;
+      const bool ok = q0 >= 0 && q1 <= total_q && L >= 0 && P >= 0 && p0 >= 0 &&
+                      (long long)p1 - p0 >= nK && P + L <= 0x7fffffffLL;
+      if (ok) {
+        d.q_start = q0;
+        d.L = (int)L;
+        d.P = P;
+        d.nKblk = (int)nK;
+        d.pt_off = p0;
+        d.nqs = (int)((L + 63) / 64);
+        units = d.nqs * Hkv * nhalves;
+      } else {
+        set_flag(err, CA_FLAG_BOUNDS);
+      }
+    }
+    int incl = units;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    int before = carry;
+    for (int w = 0; w < warp; ++w) before += warp_sum[w];
+    d.unit_start = before + incl - units;
+    if (s < num_seqs) out[s] = d;
+    __syncthreads();
+    if (tid == 0) {
+      int tot = 0;
+      for (int w = 0; w < nw; ++w) tot += warp_sum[w];
+      carry += tot;
+    }
+    __syncthreads();
+  }
+  if (tid == 0) *n_units = carry;
+}
+
 // One CTA waits on a barrier nobody arrives on, for at most limit_ns.
 __global__ void wait_probe_kernel(int32_t* err, unsigned long long limit_ns) {
   __shared__ __align__(8) uint64_t bar;
@@ -841,6 +1031,15 @@ cudaError_t launch_split_f32_bf16(const float* src, void* hi, void* lo, size_t n
   if (blocks > 148 * 16) blocks = 148 * 16;
   split_f32_bf16_kernel<<<(unsigned)blocks, 256, 0, st>>>(
       src, reinterpret_cast<__nv_bfloat16*>(hi), reinterpret_cast<__nv_bfloat16*>(lo), n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_varlen_setup(const int32_t* cu_q, const int32_t* prefix_len,
+                                const int32_t* cu_pages, int num_seqs, int total_q, int B, int Hkv,
+                                int nhalves, SeqDesc* out, int32_t* n_units, int32_t* err,
+                                cudaStream_t st) {
+  varlen_setup_kernel<<<1, 1024, 0, st>>>(cu_q, prefix_len, cu_pages, num_seqs, total_q, B, Hkv,
+                                          nhalves, out, n_units, err);
   return cudaGetLastError();
 }
 

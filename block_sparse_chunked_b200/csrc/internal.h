@@ -8,12 +8,26 @@
 
 namespace ca {
 
+// One sequence's chunk inside a chunk-attention launch.  A single-sequence
+// call carries one inline; a batch of sequences passes an array in device
+// memory, ordered as the work units are (unit_start ascending).
+struct SeqDesc {
+  int q_start;     // first row of the chunk in Q / O, and column in LSE
+  int L;           // chunk tokens
+  int P;           // prefix tokens already in the cache (any value >= 0)
+  int nKblk;       // ceil((P + L) / B): entries of its page table and table rows
+  int pt_off;      // its page table starts at page_table[pt_off]; its tables at Hkv * pt_off
+  int unit_start;  // its first work unit
+  int nqs;         // ceil(L / 64) query spans
+  int seq;         // its index in the caller's order (row of counts)
+};
+
 // Parameters of one chunk-attention launch (see chunk_attention.cu).
 struct AttnParams {
   const int32_t* page_table;
   const int32_t* tables;
   const int32_t* counts;
-  void* O;           // [L, Hq, D] bf16 or fp32 (n_splits == 1)
+  void* O;           // [L, Hq, D] bf16 or fp32 (n_splits == 1); L = all rows
   float* LSE;        // [Hq, L]                (n_splits == 1)
   float* Opart;      // [S, L, Hq, D] fp32      (n_splits > 1)
   float* LSEpart;    // [S, Hq, L] fp32         (n_splits > 1)
@@ -24,7 +38,18 @@ struct AttnParams {
   float* Osk;         // [2 * sk_ctas][NT*128][D]
   float* LSEsk;       // [2 * sk_ctas][NT*128]
   int persistent, n_units, sk_ctas;
-  int Hq, Hkv, G, HPU, nhalves, L, P, B, nPblk, nKblk, num_pages, n_splits, nqs, out_f32;
+  const int32_t* n_units_dev;  // batched calls: the exact unit count (the grid is a bound)
+  // fused mode (mask_bits != null): each CTA builds its group's table from the
+  // bit-packed masks [Hq, nQblk_mask, mask_words] instead of reading tables;
+  // one CTA per group writes it to tables_out / counts_out (either may be null)
+  const uint32_t* mask_bits;
+  int mask_words, nQblk_mask;
+  int32_t* tables_out;
+  int32_t* counts_out;
+  const SeqDesc* seqs;  // [num_seqs] in device memory, or null: one sequence, seq0
+  SeqDesc seq0;
+  int num_seqs;
+  int Hq, Hkv, G, HPU, nhalves, L, B, num_pages, n_splits, out_f32;  // L = rows of Q / O
   float scale_log2;  // log2(e) / sqrt(D)
   unsigned long long wait_ns;
 };
@@ -42,6 +67,10 @@ cudaError_t launch_sk_combine(const AttnParams& p, int D, int NT, cudaStream_t s
 cudaError_t launch_split_combine(const float* Opart, const float* LSEpart, int n_splits, int L,
                                  int Hq, int D, void* O, float* LSE, int out_f32,
                                  cudaStream_t st);
+cudaError_t launch_varlen_setup(const int32_t* cu_q, const int32_t* prefix_len,
+                                const int32_t* cu_pages, int num_seqs, int total_q, int B, int Hkv,
+                                int nhalves, SeqDesc* out, int32_t* n_units, int32_t* err,
+                                cudaStream_t st);
 cudaError_t launch_cast_f32_bf16(const float* src, void* dst, size_t n, cudaStream_t st);
 cudaError_t launch_split_f32_bf16(const float* src, void* hi, void* lo, size_t n,
                                   cudaStream_t st);

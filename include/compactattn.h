@@ -24,7 +24,9 @@
  *
  * Notation: Hq query heads, Hkv KV heads, G = Hq / Hkv heads per group; query
  * head h belongs to group h / G.  B = block = page size in tokens.
- * P = prefix_len, L = chunk_len, nQblk = L / B, nKblk = (P + L) / B.
+ * P = prefix_len, L = chunk_len, nQblk = ceil(L / B), nKblk = ceil((P + L) / B):
+ * Q-block qb holds chunk tokens [qb B, qb B + B), KV block kb holds sequence
+ * positions [kb B, kb B + B).  P and L need not be multiples of B.
  */
 #ifndef COMPACTATTN_H
 #define COMPACTATTN_H
@@ -38,7 +40,7 @@ extern "C" {
 
 #define CA_OK 0
 #define CA_ERR_ARG (-1)       /* bad shape, size or null pointer             */
-#define CA_ERR_ALIGN (-2)     /* prefix/chunk not a multiple of the block    */
+#define CA_ERR_ALIGN (-2)     /* reserved (alignment is no longer required)  */
 #define CA_ERR_DTYPE (-3)     /* unsupported dtype code                       */
 #define CA_ERR_LAUNCH (-4)    /* a CUDA launch or runtime call failed        */
 #define CA_ERR_BOUNDS (-5)    /* device: table entry or page id out of range */
@@ -122,7 +124,10 @@ size_t ca_workspace_size(int dtype, int Hq, int Hkv, int head_dim, int block, in
  *               (round to nearest even), on the device, into the workspace
  *   K_pages,
  *   V_pages     [num_pages, Hkv, B, d], dtype `dtype`; the chunk's own keys
- *               must already be in their pages
+ *               must already be in their pages, and the rows of the last
+ *               block past position P + L - 1 must hold finite values
+ *               (ca_append_kv zero-fills them): they are multiplied by zero
+ *               weights, and 0 * NaN would poison the row
  *   page_table  int32 [nKblk]: logical block -> physical page
  *   tables,
  *   counts      as written by ca_build_tables for this chunk (ascending rows)
@@ -139,14 +144,88 @@ size_t ca_workspace_size(int dtype, int Hq, int Hkv, int head_dim, int block, in
  *               on an out-of-range table entry / page id (the access is
  *               clamped, results are then undefined) or on a pipeline wait
  *               that exceeded its time limit.  Read it with ca_check().
- * Limits: head_dim in {64, 128}; block in {64, 128}; P % B == 0, L % B == 0,
- * L >= 64; Hq % Hkv == 0; num_pages >= nKblk.
+ * Limits: head_dim in {64, 128}; block in {64, 128}; P >= 0, L >= 1 (any
+ * alignment); Hq % Hkv == 0; num_pages >= nKblk.
  */
 int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, int dtype,
                        int num_pages, const int32_t* page_table, const int32_t* tables,
                        const int32_t* counts, int Hq, int Hkv, int head_dim, int block,
                        int chunk_len, int prefix_len, void* O, float* LSE, void* workspace,
                        size_t ws_bytes, int n_splits, int32_t* err_flag, void* stream);
+
+/*
+ * ca_workspace_size_varlen — bytes of device workspace for
+ * ca_chunk_attention_varlen (always > 0: it holds the per-sequence
+ * descriptors).  max_kv_len bounds P_s + L_s over the batch (it only sizes
+ * KV splits); returns (size_t)-1 for unsupported arguments.
+ */
+size_t ca_workspace_size_varlen(int dtype, int Hq, int Hkv, int head_dim, int block, int num_seqs,
+                                int total_q, int max_kv_len, int num_pages, int n_splits);
+
+/*
+ * ca_chunk_attention_varlen — ca_chunk_attention for a batch of sequences,
+ * each with its own chunk, prefix, page table and group tables, in one
+ * launch (the serving form of chunked prefill: "CompactAttention ...",
+ * Abstract, chunked prefill over an accumulated paged KV cache).
+ *
+ * Sequence s (0 <= s < num_seqs) has L_s = cu_q[s+1] - cu_q[s] chunk tokens
+ * at rows [cu_q[s], cu_q[s+1]) of Q / O (columns of LSE) and P_s =
+ * prefix_len[s] tokens already cached; its nKblk_s = ceil((P_s + L_s) / B)
+ * page-table entries are page_table[cu_pages[s] ...] and its tables
+ * [Hkv, nKblk_s] start at tables + Hkv * cu_pages[s] (ca_build_tables output
+ * for that sequence); its counts are counts[s * Hkv ...].  Every row follows
+ * the single-sequence definition above with the sequence's own P_s, tables
+ * and page table.
+ *   Q, O        [total_q, Hq, d];  LSE float32 [Hq, total_q]
+ *   K_pages,
+ *   V_pages     one page pool [num_pages, Hkv, B, d] shared by the batch
+ *   cu_q        int32 device [num_seqs + 1], cu_q[0] = 0, cu_q[num_seqs] = total_q
+ *   prefix_len  int32 device [num_seqs]
+ *   cu_pages    int32 device [num_seqs + 1]: page-table offsets,
+ *               cu_pages[s+1] - cu_pages[s] >= nKblk_s
+ *   max_kv_len  host bound on P_s + L_s (sizes KV splits)
+ *   workspace   >= ca_workspace_size_varlen(...) bytes (never NULL)
+ *   n_splits    <= 0 or 1: one CTA per (sequence, group, span, head slice);
+ *               k > 1: KV range split k ways, merged by LSE
+ * Everything runs on the stream from device arrays (capturable in a CUDA
+ * graph).  A sequence whose offsets are inconsistent is skipped (its rows
+ * are left unwritten) and CA_FLAG_BOUNDS is set in *err_flag.
+ */
+int ca_chunk_attention_varlen(const void* Q, const void* K_pages, const void* V_pages, int dtype,
+                              int num_pages, int num_seqs, int total_q, const int32_t* cu_q,
+                              const int32_t* prefix_len, int max_kv_len,
+                              const int32_t* page_table, const int32_t* cu_pages,
+                              const int32_t* tables, const int32_t* counts, int Hq, int Hkv,
+                              int head_dim, int block, void* O, float* LSE, void* workspace,
+                              size_t ws_bytes, int n_splits, int32_t* err_flag, void* stream);
+
+/*
+ * ca_chunk_attention_masked — the table builder fused into the attention
+ * prologue: ca_chunk_attention for one sequence, reading the chunk's
+ * bit-packed masks instead of prebuilt tables ("CompactAttention ...",
+ * Abstract: the per-group tables come from a Q-block union and an
+ * intra-group union of the masks).  Every CTA ORs its group's G * nQblk mask
+ * rows into a bit set in shared memory and ranks it into the ascending table
+ * (the same table ca_build_tables_bits writes), then attends exactly as
+ * ca_chunk_attention does with that table: the outputs are bit-identical.
+ *   mask_bits   uint32 [Hq, nQblk, ceil(nKblk / 32)] (device, 4-byte aligned):
+ *               bit j of word w selects KV block 32 w + j; bits past nKblk
+ *               are ignored
+ *   tables_out, counts_out  optional (may be NULL): [Hkv, nKblk] / [Hkv],
+ *               written as ca_build_tables would
+ *   workspace   >= ca_workspace_size_masked(...) bytes (may be NULL if 0)
+ *   n_splits    <= 0: automatic (KV splits when the units do not fill the
+ *               SMs); k >= 1: as for ca_chunk_attention (no persistent mode)
+ * Limits: as ca_chunk_attention, and nKblk <= 2048.
+ */
+size_t ca_workspace_size_masked(int dtype, int Hq, int Hkv, int head_dim, int block,
+                                int chunk_len, int prefix_len, int num_pages, int n_splits);
+int ca_chunk_attention_masked(const void* Q, const void* K_pages, const void* V_pages, int dtype,
+                              int num_pages, const int32_t* page_table, const uint32_t* mask_bits,
+                              int Hq, int Hkv, int head_dim, int block, int chunk_len,
+                              int prefix_len, int32_t* tables_out, int32_t* counts_out, void* O,
+                              float* LSE, void* workspace, size_t ws_bytes, int n_splits,
+                              int32_t* err_flag, void* stream);
 
 /*
  * ca_chunk_attention_noalloc — ca_chunk_attention (bf16 inputs) for callers
@@ -194,6 +273,8 @@ size_t ca_noalloc_scratch_bytes(void);
  *   K_new, V_new      [chunk_len, Hkv, head_dim], dtype `dtype`
  *   K_pages, V_pages  [num_pages, Hkv, B, head_dim], same dtype (written)
  *   page_table        int32 [ceil((prefix_len + chunk_len) / B)]
+ * The rows of the last written block after position prefix_len + chunk_len - 1
+ * are set to zero (they are read, with zero weight, by ca_chunk_attention).
  * prefix_len need not be a multiple of B; chunk_len may be 0 (then K_new and
  * V_new may be NULL and nothing is launched).  head_dim * element size must be a
  * multiple of 16 bytes; buffers 16-byte aligned.  A page id out of range sets

@@ -74,7 +74,7 @@ def _attn(bsc, **kw):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(Q=None), -1), (dict(dtype=7), -3), (dict(P=1000), -2), (dict(L=100), -2),
+    (dict(Q=None), -1), (dict(dtype=7), -3), (dict(P=-5), -1), (dict(L=0), -1),
     (dict(B=32), -1), (dict(d=96), -1), (dict(Hq=6, Hkv=4), -1), (dict(num_pages=19), -1),
     (dict(Q=ctypes.c_void_p(0x1001)), -1), (dict(dtype=1), -7), (dict(S=4), -7), (dict(S=0), -7),
 ])
@@ -99,6 +99,42 @@ def test_workspace_size_rules(bsc):
     # fp32 input adds bf16 copies of Q, K and V
     assert ws(1, 4, 1, 64, 64, 256, 1024, 20, 1) >= (256 * 4 * 64 + 2 * 20 * 64 * 64) * 2
     assert ws(0, 4, 3, 64, 64, 256, 1024, 20, 1) == ctypes.c_size_t(-1).value
+
+
+def test_workspace_size_unaligned_and_batched(bsc):
+    ws = bsc.lib.ca_workspace_size
+    # unaligned prefix / chunk: accepted (any alignment), bf16 with one split -> 0
+    assert ws(0, 32, 8, 128, 64, 100, 1000, 20, 1) == 0
+    # the chunk's blocks exceed the pages: rejected
+    assert ws(0, 32, 8, 128, 64, 100, 1000, 17, 1) == ctypes.c_size_t(-1).value
+    wv = bsc.lib.ca_workspace_size_varlen
+    # batched: descriptors always need workspace
+    n = wv(0, 32, 8, 128, 64, 5, 500, 5000, 200, 1)
+    assert 0 < n < 65536
+    # two KV splits add fp32 partials for every row
+    assert wv(0, 32, 8, 128, 64, 5, 500, 5000, 200, 2) >= 2 * 500 * 32 * 128 * 4
+    assert wv(0, 32, 8, 128, 64, 0, 500, 5000, 200, 1) == ctypes.c_size_t(-1).value
+
+
+def _varlen(bsc, **kw):
+    a = dict(Q=FAKE, K=FAKE, V=FAKE, dtype=0, num_pages=20, S=2, total_q=10, cu_q=FAKE, P=FAKE,
+             max_kv=100, pt=FAKE, cu_pages=FAKE, tables=FAKE, counts=FAKE, Hq=4, Hkv=1, d=64,
+             B=64, O=FAKE, LSE=FAKE, ws=None, wsn=0, splits=1)
+    a.update(kw)
+    return bsc.lib.ca_chunk_attention_varlen(
+        a["Q"], a["K"], a["V"], a["dtype"], a["num_pages"], a["S"], a["total_q"], a["cu_q"],
+        a["P"], a["max_kv"], a["pt"], a["cu_pages"], a["tables"], a["counts"], a["Hq"], a["Hkv"],
+        a["d"], a["B"], a["O"], a["LSE"], a["ws"], a["wsn"], a["splits"], None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(cu_q=None), -1), (dict(dtype=2), -3), (dict(S=0), -1), (dict(B=32), -1),
+    (dict(d=96), -1), (dict(Hq=6, Hkv=4), -1), (dict(total_q=-1), -1),
+    (dict(Q=ctypes.c_void_p(0x1004)), -1), (dict(), -7),
+])
+def test_varlen_rejects_bad_arguments(bsc, kw, code):
+    assert _varlen(bsc, **kw) == code
+    assert "ca_chunk_attention_varlen" in bsc.last_error()
 
 
 def test_check_and_probe_reject_null(bsc):
@@ -127,3 +163,31 @@ def _append(bsc, **kw):
 def test_append_kv_rejects_bad_arguments(bsc, kw, code):
     assert _append(bsc, **kw) == code
     assert "ca_append_kv" in bsc.last_error()
+
+
+def _masked(bsc, **kw):
+    a = dict(Q=FAKE, K=FAKE, V=FAKE, dtype=0, num_pages=40, pt=FAKE, bits=FAKE, Hq=8, Hkv=2,
+             d=128, B=64, L=256, P=1024, t=None, c=None, O=FAKE, LSE=FAKE, ws=None, wsn=0,
+             splits=1)
+    a.update(kw)
+    return bsc.lib.ca_chunk_attention_masked(
+        a["Q"], a["K"], a["V"], a["dtype"], a["num_pages"], a["pt"], a["bits"], a["Hq"],
+        a["Hkv"], a["d"], a["B"], a["L"], a["P"], a["t"], a["c"], a["O"], a["LSE"], a["ws"],
+        a["wsn"], a["splits"], None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(bits=None), -1), (dict(dtype=9), -3), (dict(P=200000, num_pages=5000), -1),
+    (dict(num_pages=10), -1), (dict(bits=ctypes.c_void_p(0x1002)), -1), (dict(L=0), -1),
+    (dict(splits=4), -7),
+])
+def test_masked_rejects_bad_arguments(bsc, kw, code):
+    assert _masked(bsc, **kw) == code
+    assert "ca_chunk_attention_masked" in bsc.last_error()
+
+
+def test_workspace_size_masked(bsc):
+    wm = bsc.lib.ca_workspace_size_masked
+    assert wm(0, 32, 8, 128, 64, 2048, 129024, 2048, 0) == 0           # 256 units: one CTA each
+    assert wm(0, 8, 2, 128, 64, 512, 1024, 24, 0) > 0                  # 16 units: KV splits
+    assert wm(0, 32, 8, 128, 64, 2048, 129024 + 64, 2049, 0) == ctypes.c_size_t(-1).value

@@ -1,0 +1,184 @@
+"""GPU parity for unaligned prefix / chunk lengths and for batches of
+sequences (ca_chunk_attention with any P, L; ca_chunk_attention_varlen)
+against the float64 oracle, plus the append -> build -> attend flow over
+ragged chunks.  Tolerances as for the aligned path: |O| <= 1e-2, |LSE| <= 1e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+O_TOL = 1e-2
+LSE_TOL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def bsc():
+    import block_sparse_chunked_b200
+    return block_sparse_chunked_b200
+
+
+def compare(O, L, Oo, Lo):
+    assert np.array_equal(np.isneginf(L), np.isneginf(Lo))
+    fin = np.isfinite(Lo)
+    if fin.any():
+        assert np.abs(L[fin] - Lo[fin]).max() <= LSE_TOL
+    assert np.abs(O - Oo).max() <= O_TOL
+
+
+def _np64(t):
+    return t.double().numpy()
+
+
+UNALIGNED = [
+    # Hq, Hkv, d, B, P, L, dtype, n_splits
+    (8, 2, 128, 64, 1000, 100, "bf16", 1),
+    (8, 2, 128, 64, 0, 1, "bf16", 1),
+    (8, 2, 128, 64, 63, 65, "bf16", 0),
+    (8, 2, 128, 64, 4097, 300, "bf16", 3),
+    (8, 2, 64, 128, 200, 77, "bf16", 1),
+    (8, 2, 128, 128, 129, 383, "bf16", 0),
+    (4, 1, 64, 64, 1000, 130, "fp32", 1),
+    (8, 8, 128, 64, 31, 33, "bf16", 1),
+]
+
+
+@pytest.mark.parametrize("Hq,Hkv,d,B,P,L,dtype,S", UNALIGNED)
+def test_unaligned_single_sequence(bsc, Hq, Hkv, d, B, P, L, dtype, S):
+    w = workloads.Workload("u", Hq, Hkv, d, dtype, P, L, B, "vslash", rho=0.1, corr=0.5,
+                           window=4, seed=P + L)
+    x = workloads.make_qkv_pages(w)
+    m = workloads.mask_for(w)
+    tables, counts = bsc.build_tables(torch.from_numpy(m).cuda(), Hkv)
+    to, co = oracle.oracle_tables(m, Hkv)
+    assert np.array_equal(tables.cpu().numpy(), to) and np.array_equal(counts.cpu().numpy(), co)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O, Lse = bsc.chunk_attention(x["Q"].cuda(), x["K_pages"].cuda(), x["V_pages"].cuda(),
+                                 x["page_table"].cuda(), tables, counts, P, n_splits=S,
+                                 err_flag=err)
+    bsc.check(err)
+    Oo, Lo = oracle.oracle_chunk_attention(_np64(x["Q"]), _np64(x["K_pages"]),
+                                           _np64(x["V_pages"]), x["page_table"].numpy(), to, co, P)
+    compare(O.float().cpu().numpy(), Lse.cpu().numpy(), Oo, Lo)
+
+
+def make_batch(seqs, Hq=8, Hkv=2, d=128, B=64, seed=0, short_pages_of=None):
+    """Sequences (P, L) over one shuffled page pool, with masks and tables per sequence."""
+    rng = np.random.default_rng(seed)
+    nKs = [-(-(P + L) // B) for P, L in seqs]
+    num_pages = sum(nKs) + 5
+    perm = rng.permutation(num_pages).astype(np.int32)
+    Kp = torch.from_numpy(rng.standard_normal((num_pages, Hkv, B, d), dtype=np.float32)).bfloat16()
+    Vp = torch.from_numpy(rng.standard_normal((num_pages, Hkv, B, d), dtype=np.float32)).bfloat16()
+    cu_q = np.concatenate([[0], np.cumsum([L for _, L in seqs])]).astype(np.int32)
+    cu_pages = np.concatenate([[0], np.cumsum(nKs)]).astype(np.int32)
+    Q = torch.from_numpy(rng.standard_normal((int(cu_q[-1]), Hq, d), dtype=np.float32)).bfloat16()
+    masks = []
+    for s, (P, L) in enumerate(seqs):
+        w = workloads.Workload("b", Hq, Hkv, d, "bf16", P, max(L, 1), B, "vslash", rho=0.1,
+                               corr=0.5, window=4, seed=seed * 100 + s)
+        masks.append(workloads.mask_for(w) if L > 0 else None)
+    if short_pages_of is not None:  # one sequence's page-table span made too short
+        cu_pages_dev = cu_pages.copy()
+        cu_pages_dev[short_pages_of + 1:] -= 1
+    else:
+        cu_pages_dev = cu_pages
+    return dict(seqs=seqs, nKs=nKs, perm=perm, Kp=Kp, Vp=Vp, cu_q=cu_q, cu_pages=cu_pages,
+                cu_pages_dev=cu_pages_dev, Q=Q, masks=masks, Hkv=Hkv, B=B)
+
+
+def run_batch(bsc, b, n_splits=1):
+    Hkv = b["Hkv"]
+    flat = torch.full((Hkv * int(b["cu_pages"][-1]),), -1, dtype=torch.int32, device="cuda")
+    counts = torch.zeros(len(b["seqs"]), Hkv, dtype=torch.int32, device="cuda")
+    for s, m in enumerate(b["masks"]):
+        if m is None:
+            continue
+        p0, nK = int(b["cu_pages"][s]), b["nKs"][s]
+        t = flat[Hkv * p0:Hkv * (p0 + nK)].view(Hkv, nK)
+        bsc.build_tables(torch.from_numpy(m).cuda(), Hkv, t, counts[s])
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    max_kv = max(P + L for P, L in b["seqs"])
+    # the page table as the device sees it follows cu_pages_dev (possibly short)
+    pt_dev = torch.from_numpy(b["perm"][:int(b["cu_pages"][-1])]).cuda()
+    O, L = bsc.chunk_attention_varlen(
+        b["Q"].cuda(), b["Kp"].cuda(), b["Vp"].cuda(), torch.from_numpy(b["cu_q"]).cuda(),
+        torch.tensor([P for P, _ in b["seqs"]], dtype=torch.int32, device="cuda"), pt_dev,
+        torch.from_numpy(b["cu_pages_dev"]).cuda(), flat, counts, max_kv, n_splits=n_splits,
+        err_flag=err)
+    return O, L, flat.cpu().numpy(), counts.cpu().numpy(), err
+
+
+def batch_oracle(b, flat, counts):
+    return oracle.oracle_varlen(_np64(b["Q"]), _np64(b["Kp"]), _np64(b["Vp"]), b["cu_q"],
+                                [P for P, _ in b["seqs"]], b["perm"][:int(b["cu_pages"][-1])],
+                                b["cu_pages"], flat, counts)
+
+
+BATCHES = [
+    [(1000, 100), (0, 1), (63, 65), (4096, 300), (130, 0)],
+    [(0, 256), (64, 64), (129, 511)],
+    [(5000, 7)] * 6,
+]
+
+
+@pytest.mark.parametrize("bi", range(len(BATCHES)))
+@pytest.mark.parametrize("n_splits", [1, 2])
+def test_varlen_batch(bsc, bi, n_splits):
+    b = make_batch(BATCHES[bi], seed=bi)
+    O, L, flat, counts, err = run_batch(bsc, b, n_splits)
+    bsc.check(err)
+    Oo, Lo = batch_oracle(b, flat, counts)
+    compare(O.float().cpu().numpy(), L.cpu().numpy(), Oo, Lo)
+
+
+def test_varlen_short_page_span_is_flagged(bsc):
+    """A sequence whose page-table span is shorter than its blocks is skipped and
+    flagged; the other sequences are still exact."""
+    b = make_batch([(300, 50), (1000, 90), (70, 40)], seed=7, short_pages_of=2)
+    O, L, flat, counts, err = run_batch(bsc, b)
+    with pytest.raises(bsc.CompactAttnError):
+        bsc.check(err)
+    Oo, Lo = batch_oracle(b, flat, counts)
+    q1 = int(b["cu_q"][2])  # rows of sequences 0 and 1
+    compare(O.float().cpu().numpy()[:q1], L.cpu().numpy()[:, :q1], Oo[:q1], Lo[:, :q1])
+
+
+def test_ragged_chunked_prefill_flow(bsc):
+    """append -> build -> attend over chunks of ragged lengths, each chunk checked
+    against the oracle on the oracle-appended cache."""
+    Hq, Hkv, d, B = 8, 2, 128, 64
+    lens = [100, 37, 64, 250, 1]
+    T = sum(lens)
+    nK_all = -(-T // B)
+    rng = np.random.default_rng(21)
+    num_pages = nK_all + 4
+    pt = torch.from_numpy(rng.permutation(num_pages)[:nK_all].astype(np.int32))
+    # stale, non-zero cache content everywhere before the first append
+    K = torch.from_numpy(rng.standard_normal((num_pages, Hkv, B, d), dtype=np.float32)).bfloat16()
+    V = torch.from_numpy(rng.standard_normal((num_pages, Hkv, B, d), dtype=np.float32)).bfloat16()
+    Kd, Vd, ptd = K.cuda(), V.cuda(), pt.cuda()
+    Ko, Vo = K.clone(), V.clone()
+    P = 0
+    for ci, Lc in enumerate(lens):
+        kn = torch.from_numpy(rng.standard_normal((Lc, Hkv, d), dtype=np.float32)).bfloat16()
+        vn = torch.from_numpy(rng.standard_normal((Lc, Hkv, d), dtype=np.float32)).bfloat16()
+        q = torch.from_numpy(rng.standard_normal((Lc, Hq, d), dtype=np.float32)).bfloat16()
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        bsc.append_kv(kn.cuda(), vn.cuda(), Kd, Vd, ptd, P, err_flag=err)
+        Ko, Vo = oracle.oracle_append_kv(Ko, Vo, pt, kn, vn, P)
+        w = workloads.Workload("f", Hq, Hkv, d, "bf16", P, Lc, B, "vslash", rho=0.2, corr=0.5,
+                               window=4, seed=ci)
+        m = workloads.mask_for(w)
+        t, c = bsc.build_tables(torch.from_numpy(m).cuda(), Hkv)
+        O, L = bsc.chunk_attention(q.cuda(), Kd, Vd, ptd, t, c, P, err_flag=err)
+        bsc.check(err)
+        assert torch.equal(Kd.cpu(), Ko) and torch.equal(Vd.cpu(), Vo)
+        Oo, Lo = oracle.oracle_chunk_attention(_np64(q), _np64(Ko), _np64(Vo), pt.numpy(),
+                                               t.cpu().numpy(), c.cpu().numpy(), P)
+        compare(O.float().cpu().numpy(), L.cpu().numpy(), Oo, Lo)
+        P += Lc
