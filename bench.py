@@ -141,10 +141,60 @@ def make_sets(w, nsets, dev):
     return x, sets
 
 
+def run_sweep(bsc, dev, stream, n_chunks=32):
+    """The full chunked-prefill sweep: 131072 tokens in 32 chunks of 4096 over one
+    growing paged cache (random page permutation).  Per chunk the KV append is
+    timed apart; the method's time is the table build + attention.  Chunk data
+    come from a seeded device generator; each chunk runs once, in order."""
+    import numpy as np
+    import torch
+
+    import workloads as wl
+    last = wl.sweep_chunk(n_chunks - 1)
+    nK_all, Hkv, B, d, Hq = last.nKblk, last.Hkv, last.block, last.head_dim, last.Hq
+    rng = np.random.default_rng(0)
+    pt = torch.from_numpy(rng.permutation(nK_all).astype(np.int32)).to(dev)
+    K = torch.zeros(nK_all, Hkv, B, d, dtype=torch.bfloat16, device=dev)
+    V = torch.zeros_like(K)
+    g = torch.Generator(device=dev).manual_seed(0)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    method_ms, append_ms, sel, dense = [], [], 0.0, 0.0
+    for c in range(n_chunks):
+        w = wl.sweep_chunk(c)
+        L = w.chunk_len
+        kn, vn = (torch.randn(L, Hkv, d, generator=g, device=dev).bfloat16() for _ in range(2))
+        q = torch.randn(L, Hq, d, generator=g, device=dev).bfloat16()
+        mask = torch.from_numpy(wl.mask_for(w)).to(dev)
+        tables = torch.empty(Hkv, w.nKblk, dtype=torch.int32, device=dev)
+        counts = torch.empty(Hkv, dtype=torch.int32, device=dev)
+        O = torch.empty_like(q)
+        lse = torch.empty(Hq, L, dtype=torch.float32, device=dev)
+        append_ms.append(timed_launch(stream, lambda: bsc.append_kv(kn, vn, K, V, pt, w.prefix_len,
+                                                                      err_flag=err)))
+
+        def method():
+            bsc.build_tables(mask, Hkv, tables, counts)
+            bsc.chunk_attention(q, K, V, pt, tables, counts, w.prefix_len, err_flag=err, out=O,
+                                lse=lse)
+        method_ms.append(timed_launch(stream, method))
+        sel += bsc.selected_flops(tables.cpu().numpy(), counts.cpu().numpy(), Hq, w.nPblk,
+                                  w.nQblk, B, d)
+        dense += bsc.dense_flops(Hq, w.nPblk, w.nQblk, B, d)
+    bsc.check(err)
+    tot = sum(method_ms)
+    return {"chunks": n_chunks, "tokens": n_chunks * last.chunk_len,
+            "method_total_ms": tot, "append_total_ms": sum(append_ms),
+            "selected_tflop": sel / 1e12, "dense_tflop": dense / 1e12,
+            "tflops_selected": sel / (tot * 1e-3) / 1e12,
+            "per_chunk_ms_first_last": [method_ms[0], method_ms[-1]]}
+
+
 def timed_launch(stream, fn):
     """Device time (ms) of the launches fn() makes.  A sleep kernel keeps the
     GPU busy while the host enqueues them, so the host-side call overhead of a
     lone launch does not land between the two events."""
+    import torch
+
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda._sleep(200_000)  # ~0.1 ms at the B200's clocks
     a.record(stream)
@@ -401,6 +451,29 @@ def main():
         del bb
     single_bytes = bsc.builder_bytes(1, w.Hq, w.Hkv, w.nQblk, w.nKblk)
 
+    # ---- the builder fused into the attention prologue (bit-packed masks, one launch)
+    for s_ in sets:
+        s_["bits"] = torch.from_numpy(wl.pack_mask_bits(s_["mask"].cpu().numpy()).view(np.int32)).to(dev)
+    ws_m = bsc.lib.ca_workspace_size_masked(0, w.Hq, w.Hkv, w.head_dim, w.block, w.chunk_len,
+                                             w.prefix_len, w.num_pages, 0)
+    ws_mt = torch.empty(max(ws_m, 1), dtype=torch.uint8, device=dev)
+    fused_ms = []
+    for i in range(args.warmup + 24):
+        s_ = sets[i % len(sets)]
+        t_ = timed_launch(stream, lambda: bsc.chunk_attention_masked(
+            s_["Q"], s_["K"], s_["V"], s_["pt"], s_["bits"], w.prefix_len, err_flag=err,
+            out=s_["O"], lse=s_["LSE"], workspace=ws_mt))
+        if i >= args.warmup:
+            fused_ms.append(t_)
+    bsc.check(err)
+    fused_res = {"ms": statistics.mean(fused_ms),
+                 "tflops": mean_flops / (statistics.mean(fused_ms) * 1e-3) / 1e12,
+                 "note": "ca_chunk_attention_masked: tables built in each CTA from bit-packed "
+                         "masks, one launch; compare ms_per_step (builder + attention)"}
+
+    # ---- the full chunked-prefill sweep (32 x 4096 tokens), one pass
+    sweep_res = run_sweep(bsc, dev, stream)
+
     # ---- end to end through the public API with pinned host buffers
     chunk_blocks = list(range(w.nPblk, w.nKblk))
     h_mask = torch.from_numpy(wl.mask_for(w, seed=0)).pin_memory()
@@ -479,6 +552,8 @@ def main():
             "dense_ms": dense_ms_mean, "dense_tflops": dense_flops / (dense_ms_mean * 1e-3) / 1e12,
             "speedup_vs_dense": dense_ms_mean / mean_attn,
             "table_build_bits": bits_res,
+            "sweep_131k": sweep_res,
+            "fused_step": fused_res,
             "kv_append": append_res,
             "table_build_batched": {"masks_per_launch": nb, "us": statistics.mean(bt) * 1e3,
                                     "GB/s": build_gbs, "frac_of_measured_hbm": build_gbs / hbm,
