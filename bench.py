@@ -471,6 +471,29 @@ def main():
                  "note": "ca_chunk_attention_masked: tables built in each CTA from bit-packed "
                          "masks, one launch; compare ms_per_step (builder + attention)"}
 
+    # ---- E4M3 paged cache (one byte per K/V element, one scale per page and head)
+    K8, sK8 = wl.quantize_pages_e4m3(x["K_pages"])
+    V8, sV8 = wl.quantize_pages_e4m3(x["V_pages"])
+    K8, sK8, V8, sV8 = K8.to(dev), sK8.to(dev), V8.to(dev), sV8.to(dev)
+    ws_f8 = torch.empty(bsc.lib.ca_workspace_size_fp8(w.Hq, w.Hkv, w.head_dim, w.block,
+                                                      w.chunk_len, w.prefix_len, w.num_pages, 0),
+                        dtype=torch.uint8, device=dev)
+    fp8_ms = []
+    for i in range(args.warmup + 24):
+        s_ = sets[i % len(sets)]
+        t_ = timed_launch(stream, lambda: bsc.chunk_attention_fp8(
+            s_["Q"], K8, V8, sK8, sV8, s_["pt"], s_["tables"], s_["counts"], w.prefix_len,
+            err_flag=err, out=s_["O"], lse=s_["LSE"], workspace=ws_f8))
+        if i >= args.warmup:
+            fp8_ms.append(t_)
+    bsc.check(err)
+    fp8_res = {"ms": statistics.mean(fp8_ms),
+               "tflops": mean_flops / (statistics.mean(fp8_ms) * 1e-3) / 1e12,
+               "kv_cache_bytes": 2 * K8.numel(), "bf16_kv_cache_bytes": 4 * K8.numel(),
+               "note": "ca_chunk_attention_fp8 incl. the Q cast and scale gather; one page "
+                       "buffer (not rotated)"}
+    del K8, V8
+
     # ---- the full chunked-prefill sweep (32 x 4096 tokens), one pass
     sweep_res = run_sweep(bsc, dev, stream)
 
@@ -554,6 +577,7 @@ def main():
             "table_build_bits": bits_res,
             "sweep_131k": sweep_res,
             "fused_step": fused_res,
+            "fp8_kv": fp8_res,
             "kv_append": append_res,
             "table_build_batched": {"masks_per_launch": nb, "us": statistics.mean(bt) * 1e3,
                                     "GB/s": build_gbs, "frac_of_measured_hbm": build_gbs / hbm,

@@ -28,6 +28,7 @@ from ._capi import (  # noqa: F401
     chunk_attention,
     chunk_attention_varlen,
     chunk_attention_masked,
+    chunk_attention_fp8,
     append_kv,
     check,
     wait_probe,

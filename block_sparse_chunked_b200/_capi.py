@@ -36,6 +36,10 @@ EXPORTS = {
     "ca_noalloc_scratch_bytes": (_c_size, []),
     "ca_workspace_size_varlen": (_c_size, [_c_int] * 10),
     "ca_workspace_size_masked": (_c_size, [_c_int] * 9),
+    "ca_workspace_size_fp8": (_c_size, [_c_int] * 8),
+    "ca_chunk_attention_fp8": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _vp, _vp, _c_int,
+                                        _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp,
+                                        _c_size, _c_int, _vp, _vp]),
     "ca_chunk_attention_masked": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _vp, _vp, _c_int, _c_int,
                                            _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp,
                                            _vp, _c_size, _c_int, _vp, _vp]),
@@ -197,6 +201,42 @@ def chunk_attention(Q, K_pages, V_pages, page_table, tables, counts, prefix_len,
         _ptr(Q), _ptr(K_pages), _ptr(V_pages), code, num_pages, _ptr(page_table), _ptr(tables),
         _ptr(counts), Hq, Hkv, d, B, L, prefix_len, _ptr(out), _ptr(lse),
         _ptr(workspace) if ws_n else None, ws_n, n_splits, _ptr(err_flag), _stream()))
+    return out, lse
+
+
+def chunk_attention_fp8(Q, K8, V8, K_scale, V_scale, page_table, tables, counts, prefix_len,
+                        n_splits=0, err_flag=None, out=None, lse=None, workspace=None):
+    """Chunk attention over an E4M3 paged cache: K8/V8 uint8 [num_pages, Hkv, B, d],
+    K_scale/V_scale float32 [num_pages, Hkv]; Q bf16 [L, Hq, d].  Returns O (bf16)
+    and LSE float32 [Hq, L]."""
+    _need_cuda("Q", Q, (torch.bfloat16,), 3)
+    _need_cuda("K8", K8, (torch.uint8,), 4)
+    _need_cuda("V8", V8, (torch.uint8,), 4)
+    _need_cuda("K_scale", K_scale, (torch.float32,), 2)
+    _need_cuda("V_scale", V_scale, (torch.float32,), 2)
+    _need_cuda("page_table", page_table, (torch.int32,), 1)
+    _need_cuda("tables", tables, (torch.int32,), 2)
+    _need_cuda("counts", counts, (torch.int32,), 1)
+    L, Hq, d = Q.shape
+    num_pages, Hkv, B, d2 = K8.shape
+    nK = -(-(prefix_len + L) // B)
+    if (V8.shape != K8.shape or d2 != d or tuple(K_scale.shape) != (num_pages, Hkv)
+            or tuple(V_scale.shape) != (num_pages, Hkv) or page_table.numel() < nK
+            or tables.shape[0] != Hkv or tables.shape[1] < nK or counts.numel() < Hkv):
+        raise ValueError("inconsistent shapes for chunk_attention_fp8")
+    if out is None:
+        out = torch.empty_like(Q)
+    if lse is None:
+        lse = torch.empty(Hq, L, dtype=torch.float32, device=Q.device)
+    ws_n = lib.ca_workspace_size_fp8(Hq, Hkv, d, B, L, prefix_len, num_pages, n_splits)
+    if ws_n == ctypes.c_size_t(-1).value:
+        raise CompactAttnError(CA_ERR_ARG, "invalid shapes for ca_workspace_size_fp8")
+    if workspace is None or workspace.numel() < ws_n:
+        workspace = torch.empty(ws_n, dtype=torch.uint8, device=Q.device)
+    _ok(lib.ca_chunk_attention_fp8(
+        _ptr(Q), _ptr(K8), _ptr(V8), _ptr(K_scale), _ptr(V_scale), num_pages, _ptr(page_table),
+        _ptr(tables), _ptr(counts), Hq, Hkv, d, B, L, prefix_len, _ptr(out), _ptr(lse),
+        _ptr(workspace), ws_n, n_splits, _ptr(err_flag), _stream()))
     return out, lse
 
 

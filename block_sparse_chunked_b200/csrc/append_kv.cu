@@ -20,35 +20,33 @@
 
 namespace ca {
 
+// Block (row i, head-group y): threadIdx.x = 16-byte vector of a head's row,
+// threadIdx.y = head within the block's group of heads; no index division.
 __global__ void __launch_bounds__(256)
     append_kv_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
                      uint4* __restrict__ k_pages, uint4* __restrict__ v_pages,
                      const int32_t* __restrict__ page_table, int prefix_len, int chunk_len,
-                     int Hkv, int vec_per_row, int block, int num_pages, int nKblk, int tail,
+                     int Hkv, int vec_per_row, int block, int num_pages, int nKblk,
                      int32_t* err) {
-  // 32-bit index math (the host bounds the vector count below 2^31)
-  const unsigned total = (unsigned)(chunk_len + tail) * (unsigned)Hkv * (unsigned)vec_per_row;
-  for (unsigned idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += gridDim.x * blockDim.x) {
-    const unsigned v = idx % (unsigned)vec_per_row;
-    const unsigned rg = idx / (unsigned)vec_per_row;
-    const int g = (int)(rg % (unsigned)Hkv);
-    const int i = (int)(rg / (unsigned)Hkv);
-    const int pos = prefix_len + i;
-    const int kb = pos / block;
-    int page = (kb < nKblk) ? page_table[kb] : -1;
-    if (page < 0 || page >= num_pages) {
-      if (err) atomicOr(err, CA_FLAG_BOUNDS);
-      continue;  // never write outside the cache
-    }
-    const size_t dst = (((size_t)page * Hkv + g) * block + pos % block) * vec_per_row + v;
-    if (i < chunk_len) {
-      k_pages[dst] = __ldcs(k_new + idx);
-      v_pages[dst] = __ldcs(v_new + idx);
-    } else {
-      k_pages[dst] = make_uint4(0u, 0u, 0u, 0u);
-      v_pages[dst] = make_uint4(0u, 0u, 0u, 0u);
-    }
+  const int i = blockIdx.x;  // token of the chunk, or of the cleared tail past it
+  const int g = blockIdx.y * blockDim.y + threadIdx.y;
+  const int v = threadIdx.x;
+  if (g >= Hkv) return;
+  const int pos = prefix_len + i;
+  const int kb = pos / block;
+  const int page = (kb < nKblk) ? page_table[kb] : -1;
+  if (page < 0 || page >= num_pages) {
+    if (err && v == 0) atomicOr(err, CA_FLAG_BOUNDS);
+    return;  // never write outside the cache
+  }
+  const size_t dst = (((size_t)page * Hkv + g) * block + pos % block) * vec_per_row + v;
+  if (i < chunk_len) {
+    const size_t src = ((size_t)i * Hkv + g) * vec_per_row + v;
+    k_pages[dst] = __ldcs(k_new + src);
+    v_pages[dst] = __ldcs(v_new + src);
+  } else {
+    k_pages[dst] = make_uint4(0u, 0u, 0u, 0u);
+    v_pages[dst] = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
@@ -59,14 +57,16 @@ cudaError_t launch_append_kv(const void* k_new, const void* v_new, void* k_pages
   const int vec = row_bytes / 16;
   const int end = prefix_len + chunk_len;
   const int tail = chunk_len > 0 ? (block - end % block) % block : 0;  // rest of the last block
-  const long long total = (long long)(chunk_len + tail) * Hkv * vec;
-  if (total == 0) return cudaSuccess;
-  long long blocks = (total + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
-  append_kv_kernel<<<(unsigned)blocks, 256, 0, st>>>(
+  const int rows = chunk_len + tail;
+  if (rows == 0) return cudaSuccess;
+  int hy = 256 / vec;  // heads per block
+  if (hy < 1) hy = 1;
+  if (hy > Hkv) hy = Hkv;
+  const dim3 blk(vec, hy), grid(rows, (Hkv + hy - 1) / hy);
+  append_kv_kernel<<<grid, blk, 0, st>>>(
       static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
       static_cast<uint4*>(k_pages), static_cast<uint4*>(v_pages), page_table, prefix_len,
-      chunk_len, Hkv, vec, block, num_pages, nKblk, tail, err);
+      chunk_len, Hkv, vec, block, num_pages, nKblk, err);
   return cudaGetLastError();
 }
 
@@ -96,8 +96,8 @@ extern "C" int ca_append_kv(const void* K_new, const void* V_new, int dtype, voi
     ca::set_last_error("ca_append_kv: the chunk's blocks exceed num_pages");
     return CA_ERR_ARG;
   }
-  if ((long long)(chunk_len + block) * Hkv * (head_dim * esize / 16) >= 0x7fffffffLL) {
-    ca::set_last_error("ca_append_kv: chunk too large for one call");
+  if (head_dim * esize / 16 > 256 || (long long)chunk_len + block > 0x7fffffffLL) {
+    ca::set_last_error("ca_append_kv: row or chunk too large for one call");
     return CA_ERR_ARG;
   }
   const uintptr_t al = reinterpret_cast<uintptr_t>(K_new) | reinterpret_cast<uintptr_t>(V_new) |

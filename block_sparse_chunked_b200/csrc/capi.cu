@@ -130,12 +130,12 @@ bool plan(int Hq, int Hkv, int head_dim, int block, int chunk_len, int prefix_le
 
 struct WsLayout {
   size_t opart = 0, lsepart = 0, q = 0, qlo = 0, k = 0, v = 0, sched = 0, osk = 0, lsesk = 0,
-         seqs = 0, nunits = 0, total = 0;
+         seqs = 0, nunits = 0, q16 = 0, esc = 0, total = 0;
 };
 
 // rows = rows of Q / O; num_seqs > 0 reserves the batched call's descriptors.
 WsLayout ws_layout(int dtype, int Hq, int Hkv, int D, int B, long long rows, int num_pages,
-                   const Plan& pl, int num_seqs = 0) {
+                   const Plan& pl, int num_seqs = 0, int nKblk_e4m3 = 0) {
   WsLayout w;
   size_t off = 0;
   const int S = pl.n_splits;
@@ -159,6 +159,12 @@ WsLayout ws_layout(int dtype, int Hq, int Hkv, int D, int B, long long rows, int
     off = align256(off + (size_t)S * rows * Hq * D * 4);
     w.lsepart = off;
     off = align256(off + (size_t)S * Hq * rows * 4);
+  }
+  if (dtype == CA_DTYPE_E4M3) {  // f16 copy of Q, per-entry page scales
+    w.q16 = off;
+    off = align256(off + (size_t)rows * Hq * D * 2);
+    w.esc = off;
+    off = align256(off + (size_t)Hkv * nKblk_e4m3 * 8);
   }
   if (dtype == CA_DTYPE_FP32) {
     w.q = off;
@@ -272,6 +278,7 @@ int run_attention(const char* who, const void* Q, const void* K_pages, const voi
                   int dtype, int num_pages, int Hq, int Hkv, int D, int B, int rows,
                   const Plan& pl, const WsLayout& wl, uint8_t* ws, int grid, AttnParams& p,
                   cudaStream_t st) {
+  const bool kv8 = dtype == CA_DTYPE_E4M3;  // Q is then already the f16 copy
   EncodeTiledFn enc = encoder();
   if (!enc) return fail(CA_ERR_LAUNCH, "%s: cuTensorMapEncodeTiled unavailable", who);
   const void* q = Q;
@@ -305,21 +312,27 @@ int run_attention(const char* who, const void* Q, const void* K_pages, const voi
     cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
     cuuint32_t box[3] = {64, 1, 64};
     cuuint32_t es[3] = {1, 1, 1};
-    CUresult r = enc(which ? &tqlo : &tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+    CUresult r = enc(which ? &tqlo : &tq,
+                     kv8 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                      const_cast<void*>(which ? qlo : q), dims, strides, box, es,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(CA_ERR_LAUNCH, "%s: tensor map (Q) encode failed: %d", who, (int)r);
   }
   for (int which = 0; which < 2; ++which) {
+    // bf16 pages: 64-element boxes with the 128-byte swizzle the MMAs read;
+    // E4M3 pages: whole rows of D bytes, unswizzled, into the staging area
+    const int esz = kv8 ? 1 : 2;
     cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)B, (cuuint64_t)Hkv, (cuuint64_t)num_pages};
-    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)B * D * 2,
-                             (cuuint64_t)Hkv * B * D * 2};
-    cuuint32_t box[4] = {64, (cuuint32_t)B, 1, 1};
+    cuuint64_t strides[3] = {(cuuint64_t)D * esz, (cuuint64_t)B * D * esz,
+                             (cuuint64_t)Hkv * B * D * esz};
+    cuuint32_t box[4] = {kv8 ? (cuuint32_t)D : 64u, (cuuint32_t)B, 1, 1};
     cuuint32_t es[4] = {1, 1, 1, 1};
-    CUresult r = enc(which ? &tv : &tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+    CUresult r = enc(which ? &tv : &tk,
+                     kv8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                      const_cast<void*>(which ? vp : kp), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     kv8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
       return fail(CA_ERR_LAUNCH, "%s: tensor map (%s pages) encode failed: %d", who,
@@ -343,10 +356,11 @@ int run_attention(const char* who, const void* Q, const void* K_pages, const voi
   p.B = B;
   p.num_pages = num_pages;
   p.n_splits = pl.n_splits;
-  p.out_f32 = dtype == CA_DTYPE_FP32 ? 1 : 0;
+  p.out_f32 = dtype == CA_DTYPE_FP32 ? 1 : 0;  // E4M3 pages: O is bf16
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   p.wait_ns = kWaitNs;
-  e = launch_chunk_attention(tq, tqlo, tk, tv, p, D, pl.NT, dtype == CA_DTYPE_FP32, grid, st);
+  e = launch_chunk_attention(tq, tqlo, tk, tv, p, D, pl.NT, dtype == CA_DTYPE_FP32, kv8, grid,
+                             st);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   if (pl.persistent) {
     e = launch_sk_combine(p, D, pl.NT, st);
@@ -405,12 +419,12 @@ int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, 
 }
 
 namespace {
-// Fused calls: one CTA per unit (the table is built per CTA), KV splits when
+// Fused and E4M3 calls: one CTA per unit (no persistent grid), KV splits when
 // the units do not fill the SMs.
 bool plan_masked(int Hq, int Hkv, int head_dim, int block, int chunk_len, int prefix_len,
-                 int n_splits, Plan& pl, SeqDesc& d) {
+                 int n_splits, Plan& pl, SeqDesc& d, int max_nKblk = 2048) {
   if (!plan(Hq, Hkv, head_dim, block, chunk_len, prefix_len, 1, pl, d)) return false;
-  if (d.nKblk > 2048) return false;
+  if (d.nKblk > max_nKblk) return false;
   const int max_stages = (d.nKblk + pl.spb - 1) / pl.spb;
   int S = n_splits;
   if (S <= 0) S = pl.units >= kSMs ? 1 : (2 * kSMs + pl.units - 1) / pl.units;
@@ -473,6 +487,64 @@ int ca_chunk_attention_masked(const void* Q, const void* K_pages, const void* V_
   return run_attention(who, Q, K_pages, V_pages, dtype, num_pages, Hq, Hkv, head_dim, block,
                        chunk_len, pl, wl, static_cast<uint8_t*>(workspace),
                        pl.units * pl.n_splits, p, static_cast<cudaStream_t>(stream));
+}
+
+size_t ca_workspace_size_fp8(int Hq, int Hkv, int head_dim, int block, int chunk_len,
+                             int prefix_len, int num_pages, int n_splits) {
+  Plan pl;
+  SeqDesc d;
+  if (!plan_masked(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl, d, 1 << 30))
+    return (size_t)-1;
+  if (num_pages < d.nKblk) return (size_t)-1;
+  return ws_layout(CA_DTYPE_E4M3, Hq, Hkv, head_dim, block, chunk_len, num_pages, pl, 0, d.nKblk)
+      .total;
+}
+
+int ca_chunk_attention_fp8(const void* Q, const uint8_t* K_pages, const uint8_t* V_pages,
+                           const float* K_scale, const float* V_scale, int num_pages,
+                           const int32_t* page_table, const int32_t* tables,
+                           const int32_t* counts, int Hq, int Hkv, int head_dim, int block,
+                           int chunk_len, int prefix_len, void* O, float* LSE, void* workspace,
+                           size_t ws_bytes, int n_splits, int32_t* err_flag, void* stream) {
+  const char* who = "ca_chunk_attention_fp8";
+  if (!Q || !K_pages || !V_pages || !K_scale || !V_scale || !page_table || !tables || !counts ||
+      !O || !LSE)
+    return fail(CA_ERR_ARG, "%s: null pointer", who);
+  Plan pl;
+  SeqDesc d;
+  if (!plan_masked(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl, d, 1 << 30))
+    return fail(CA_ERR_ARG,
+                "%s: unsupported shape Hq=%d Hkv=%d head_dim=%d block=%d chunk_len=%d "
+                "prefix_len=%d",
+                who, Hq, Hkv, head_dim, block, chunk_len, prefix_len);
+  if (num_pages < d.nKblk)
+    return fail(CA_ERR_ARG, "%s: num_pages=%d < nKblk=%d", who, num_pages, d.nKblk);
+  if (!aligned16(Q) || !aligned16(K_pages) || !aligned16(V_pages) || !aligned16(O))
+    return fail(CA_ERR_ARG, "%s: Q, K_pages, V_pages and O must be 16-byte aligned", who);
+  const WsLayout wl =
+      ws_layout(CA_DTYPE_E4M3, Hq, Hkv, head_dim, block, chunk_len, num_pages, pl, 0, d.nKblk);
+  if (!workspace || ws_bytes < wl.total || !aligned16(workspace))
+    return fail(CA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, got %zu", who, wl.total,
+                workspace ? ws_bytes : (size_t)0);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaError_t e = launch_cast_bf16_f16(Q, ws + wl.q16, (size_t)chunk_len * Hq * head_dim, st);
+  if (e == cudaSuccess)
+    e = launch_gather_scales(tables, counts, page_table, K_scale, V_scale, Hkv, d.nKblk,
+                             num_pages, reinterpret_cast<float2*>(ws + wl.esc), err_flag, st);
+  if (e != cudaSuccess) return cuda_fail(e, "ca_chunk_attention_fp8 prologue launch");
+  AttnParams p{};
+  p.page_table = page_table;
+  p.tables = tables;
+  p.counts = counts;
+  p.O = O;
+  p.LSE = LSE;
+  p.err = err_flag;
+  p.escale = reinterpret_cast<const float2*>(ws + wl.esc);
+  p.seq0 = d;
+  p.num_seqs = 1;
+  return run_attention(who, ws + wl.q16, K_pages, V_pages, CA_DTYPE_E4M3, num_pages, Hq, Hkv,
+                       head_dim, block, chunk_len, pl, wl, ws, pl.units * pl.n_splits, p, st);
 }
 
 int ca_chunk_attention_varlen(const void* Q, const void* K_pages, const void* V_pages, int dtype,

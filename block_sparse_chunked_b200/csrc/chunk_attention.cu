@@ -33,6 +33,8 @@
 // and unwinds instead of hanging.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -54,25 +56,34 @@ __device__ __forceinline__ void set_flag(int32_t* err, int f) {
 // QSPLIT: Q is given as two bf16 terms (hi + lo) of an fp32 input and
 // S = Q_hi K^T + Q_lo K^T, which removes the rounding error of Q (the error
 // term shared by all keys of a row); used for fp32 inputs.
-template <int D, int NT, bool QSPLIT>
+//
+// KV8: K/V pages hold E4M3 bytes; TMA brings a stage's K and V bytes into a
+// staging area, warps 2-3 widen them to f16 into the swizzled operand ring, and
+// the MMAs run kind::f16 with f16 operands (Q converted to f16, P written as
+// f16).  The per-page scales are applied in the softmax.
+template <int D, int NT, bool QSPLIT, bool KV8 = false>
 struct Smem {
   static constexpr int kQTerms = QSPLIT ? 2 : 1;
-  static constexpr int kChunkBytes = 128 * 128;         // 128 rows x 128 B (64 bf16)
+  static constexpr int kChunkBytes = 128 * 128;         // 128 rows x 128 B (64 16-bit)
   static constexpr int kQTile = 128 * D * 2;            // one 128-row Q tile
   static constexpr int kKV = kStageKeys * D * 2;        // one stage of K (or V)
+  static constexpr int kStg = KV8 ? 2 * kStageKeys * D : 0;  // E4M3 K + V of one stage
   // K/V ring depth: two stages unless the split Q tiles leave room for one only
-  static constexpr int kNS = (kQTerms * NT * kQTile + 4 * kKV <= 200 * 1024) ? 2 : 1;
+  static constexpr int kNS =
+      KV8 ? 2 : ((kQTerms * NT * kQTile + 4 * kKV <= 200 * 1024) ? 2 : 1);
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQTerms * NT * kQTile;
   static constexpr int kVOff = kKOff + kNS * kKV;
-  static constexpr int kBarOff = kVOff + kNS * kKV;
+  static constexpr int kStgOff = kVOff + kNS * kKV;
+  static constexpr int kBarOff = kStgOff + kStg;
   // barriers: q_full, full_k[NS], full_v[NS], empty_k[NS], empty_v[NS],
-  //           s_full[2], p_full[2], o_done, drain, q_free
-  static constexpr int kNumBars = 1 + 4 * kNS + 2 + 2 + 3;
+  //           s_full[2], p_full[2], o_done, drain, q_free (+ stg_full, stg_empty)
+  static constexpr int kNumBars = 1 + 4 * kNS + 2 + 2 + 3 + (KV8 ? 2 : 0);
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   // persistent schedule: per-unit live entries, prefix of stage counts, warp sums
+  // (not used with E4M3 pages, which run one CTA per unit or KV splits)
   static constexpr int kSchedOff = kMiscOff + 64;
-  static constexpr int kBytes = kSchedOff + (2 * 2048 + 1 + 32) * 4;
+  static constexpr int kBytes = kSchedOff + (KV8 ? 0 : (2 * 2048 + 1 + 32) * 4);
   static constexpr int kAlloc = kBytes + 1024;          // slack for 1024-B alignment
 };
 
@@ -219,13 +230,13 @@ __device__ int fused_group_table(const AttnParams& p, const UnitCoord& uc, int32
 // How a piece's result leaves the CTA.
 enum PieceOut : int { kOutFinal = 0, kOutSplit = 1, kOutSK = 2 };
 
-template <int D, int NT, bool QSPLIT>
+template <int D, int NT, bool QSPLIT, bool KV8>
 __global__ void __launch_bounds__(128 + NT * 128, 1)
     chunk_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmQlo,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using S = Smem<D, NT, QSPLIT>;
+  using S = Smem<D, NT, QSPLIT, KV8>;
   constexpr int kNS = S::kNS;
   constexpr int KCH = D / 64;  // 64-element (128-byte) chunks along head_dim
   extern __shared__ uint8_t smem_raw[];
@@ -243,6 +254,8 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
   const uint32_t o_done = bars + 8u * (5 + 4 * kNS);
   const uint32_t drain = bars + 8u * (6 + 4 * kNS);
   const uint32_t q_free = bars + 8u * (7 + 4 * kNS);
+  const uint32_t stg_full = bars + 8u * (8 + 4 * kNS);   // KV8 only
+  const uint32_t stg_empty = bars + 8u * (9 + 4 * kNS);  // KV8 only
   int* misc = reinterpret_cast<int*>(sm + S::kMiscOff);
   // misc[0] tmem base, [1] live entries (one-piece mode), [2] first stage,
   // [3] last stage (exclusive), [4] live entries of the fused table (thread 0
@@ -328,8 +341,8 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
     mbar_init(q_full, 1);
     mbar_init(q_free, 1);
     for (int s = 0; s < kNS; ++s) {
-      mbar_init(full_k(s), 1);
-      mbar_init(full_v(s), 1);
+      mbar_init(full_k(s), KV8 ? 2 : 1);  // KV8: the two widening warps arrive
+      mbar_init(full_v(s), KV8 ? 2 : 1);
       mbar_init(empty_k(s), 1);
       mbar_init(empty_v(s), 1);
     }
@@ -339,6 +352,10 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
     }
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
+    if (KV8) {
+      mbar_init(stg_full, 1);
+      mbar_init(stg_empty, 2);
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -446,6 +463,22 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
           }
           page[pi] = __shfl_sync(0xffffffffu, pg_cache, e - cache_base);
         }
+        if (KV8) {
+          // E4M3 bytes of the stage's pages into the staging area, once the
+          // widening warps have finished with the previous stage's bytes
+          if (gj > 0) ok = wait_warp(stg_empty, (gj - 1) & 1, p, abort_flag);
+          if (ok) {
+            const uint32_t b8 = (uint32_t)npg * p.B * D;
+            mbar_expect_tx_w(stg_full, 2 * b8);
+            for (int pi = 0; pi < npg; ++pi)
+              tma_load_4d_w(sbase + S::kStgOff + pi * p.B * D, &tmK, stg_full, 0, 0, uc.g,
+                            page[pi], pol);
+            for (int pi = 0; pi < npg; ++pi)
+              tma_load_4d_w(sbase + S::kStgOff + kStageKeys * D + pi * p.B * D, &tmV, stg_full,
+                            0, 0, uc.g, page[pi], pol);
+          }
+          continue;
+        }
         if (round > 0) ok = wait_warp(empty_k(slot), (round - 1) & 1, p, abort_flag);
         if (ok) {
           mbar_expect_tx_w(full_k(slot), bytes);
@@ -467,9 +500,13 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
     });
     if (lane == 0) {
       // Do not leave with copies in flight: the last stages' loads must land.
-      for (int G = max(0, gj - kNS); G < gj; ++G) {
-        mbar_wait(full_k(G % kNS), (G / kNS) & 1, p.wait_ns);
-        mbar_wait(full_v(G % kNS), (G / kNS) & 1, p.wait_ns);
+      if (KV8) {
+        if (gj > 0) mbar_wait(stg_full, (gj - 1) & 1, p.wait_ns);
+      } else {
+        for (int G = max(0, gj - kNS); G < gj; ++G) {
+          mbar_wait(full_k(G % kNS), (G / kNS) & 1, p.wait_ns);
+          mbar_wait(full_v(G % kNS), (G / kNS) & 1, p.wait_ns);
+        }
       }
       if (pn > 0) mbar_wait(q_full, (pn - 1) & 1, p.wait_ns);
     }
@@ -480,9 +517,9 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
     // Descriptors differ per MMA only in the start-address field (address >> 4
     // in bits 0-13): build each operand's descriptor once and add the
     // compile-time byte offset >> 4 per K-step.
-    constexpr uint32_t kIdescPV = idesc_bf16(128, D, 1);
-    constexpr uint32_t kIdescS128 = idesc_bf16(128, 128, 0);
-    constexpr uint32_t kIdescS64 = idesc_bf16(128, 64, 0);
+    constexpr uint32_t kIdescPV = KV8 ? idesc_f16(128, D, 1) : idesc_bf16(128, D, 1);
+    constexpr uint32_t kIdescS128 = KV8 ? idesc_f16(128, 128, 0) : idesc_bf16(128, 128, 0);
+    constexpr uint32_t kIdescS64 = KV8 ? idesc_f16(128, 64, 0) : idesc_bf16(128, 64, 0);
     uint64_t qdesc[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) qdesc[t] = smem_desc_sw128(sbase + S::kQOff + t * S::kQTile, 16, 1024);
@@ -574,6 +611,57 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
     // every MMA issued by this warp has finished before TMEM is released
     mma_commit_w(drain);
     mbar_wait(drain, 0, p.wait_ns);
+  } else if (KV8 && (warp == 2 || warp == 3)) {
+    // ================================================================ E4M3 -> f16
+    // Widen the staged bytes of each stage into the swizzled f16 operand ring
+    // (same layout the TMA gives bf16 pages: 64-element chunks of 128 rows x
+    // 128 B, 16-byte units XOR-swizzled by row), K then V.
+    const int ct = threadIdx.x - 64;  // 0 .. 63
+    int gj = 0;
+    bool ok = true;
+    auto widen = [&](uint32_t src_off, uint32_t dst_off, int rows) {
+      constexpr int CPR = D / 16;  // 16-byte chunks per E4M3 row
+      const uint8_t* src = sm + src_off;
+      uint8_t* dst = sm + dst_off;
+      for (int i = ct; i < rows * CPR; i += 64) {
+        const int r = i / CPR, q = i % CPR;
+        const uint4 x = *reinterpret_cast<const uint4*>(src + r * D + q * 16);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t h[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] & 0xffffu), __NV_E4M3);
+          const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] >> 16), __NV_E4M3);
+          h[2 * k] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
+          h[2 * k + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
+        }
+        const int u = (q & 3) * 2;  // first 16-byte unit of these 16 elements in their row
+        uint8_t* rowp = dst + (q >> 2) * S::kChunkBytes + r * 128;
+        *reinterpret_cast<uint4*>(rowp + ((u ^ (r & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4*>(rowp + (((u + 1) ^ (r & 7)) << 4)) =
+            make_uint4(h[4], h[5], h[6], h[7]);
+      }
+      fence_proxy_async_smem();  // the tensor cores read these bytes next
+      __syncwarp();
+    };
+    for_each_piece([&](int, int live, int s0, int s1, int, int) {
+      for (int stage = s0; stage < s1 && ok; ++stage, ++gj) {
+        const int slot = gj % kNS, round = gj / kNS;
+        const int rows = min(spb, live - stage * spb) * p.B;
+        ok = wait_warp(stg_full, gj & 1, p, abort_flag);
+        if (ok && round > 0) ok = wait_warp(empty_k(slot), (round - 1) & 1, p, abort_flag);
+        if (!ok) break;
+        widen(S::kStgOff, S::kKOff + slot * S::kKV, rows);
+        if (lane == 0) mbar_arrive(full_k(slot));
+        if (round > 0) ok = wait_warp(empty_v(slot), (round - 1) & 1, p, abort_flag);
+        if (!ok) break;
+        widen(S::kStgOff + kStageKeys * D, S::kVOff + slot * S::kKV, rows);
+        if (lane == 0) {
+          mbar_arrive(full_v(slot));
+          mbar_arrive(stg_empty);
+        }
+      }
+    });
   } else if (warp >= 4) {
     // ================================================================ softmax / epilogue
     const int t = (warp - 4) >> 2;
@@ -611,6 +699,12 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
         const int npg = min(spb, live - stage * spb);
         const int nvalid = npg * p.B;
         const bool mask_stage = stage * spb + npg > mask_e;
+        float2 scl_a = make_float2(1.f, 1.f), scl_b = scl_a;  // KV8: (K, V) scales per half
+        if (KV8) {
+          const float2* es = p.escale + (size_t)uc.g * uc.d.nKblk + stage * spb;
+          scl_a = es[0];
+          scl_b = npg > 1 ? es[1] : scl_a;
+        }
         ok = wait_warp(s_full(t), G & 1, p, abort_flag);
         if (!ok) break;
         tc_fence_after();
@@ -635,14 +729,35 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
             if (c >= cm0 && (c - cm0) > lim) sr[c] = -INFINITY;
         }
         // row max of the raw scores (scale > 0 commutes with max)
-        float mx0 = max3(sr[0], sr[1], sr[2]);
-        float mx1 = max3(sr[3], sr[4], sr[5]);
+        float mx;
+        float scA = p.scale_log2, scB = p.scale_log2, lbA = 0.f, lbB = 0.f;
+        if (KV8) {
+          // E4M3 pages: the log2-domain score of a key of page P is
+          // s * scale * sK_P, and its weight enters PV multiplied by sV_P, so the
+          // exponent carries + log2(sV_P) (the row sum divides it out again)
+          scA *= scl_a.x;
+          scB *= scl_b.x;
+          lbA = __log2f(scl_a.y);
+          lbB = __log2f(scl_b.y);
+          float ha = max3(sr[0], sr[1], sr[2]), hb = max3(sr[64], sr[65], sr[66]);
 #pragma unroll
-        for (int c = 6; c < kStageKeys - 2; c += 4) {
-          mx0 = max3(mx0, sr[c], sr[c + 1]);
-          mx1 = max3(mx1, sr[c + 2], sr[c + 3]);
+          for (int c = 3; c < 63; c += 2) {
+            ha = max3(ha, sr[c], sr[c + 1]);
+            hb = max3(hb, sr[64 + c], sr[64 + c + 1]);
+          }
+          ha = fmaxf(ha, sr[63]);
+          hb = fmaxf(hb, sr[127]);
+          mx = fmaxf(ha * scA + lbA, hb * scB + lbB);
+        } else {
+          float mx0 = max3(sr[0], sr[1], sr[2]);
+          float mx1 = max3(sr[3], sr[4], sr[5]);
+#pragma unroll
+          for (int c = 6; c < kStageKeys - 2; c += 4) {
+            mx0 = max3(mx0, sr[c], sr[c + 1]);
+            mx1 = max3(mx1, sr[c + 2], sr[c + 3]);
+          }
+          mx = max3(mx0, mx1, fmaxf(sr[kStageKeys - 2], sr[kStageKeys - 1])) * p.scale_log2;
         }
-        const float mx = max3(mx0, mx1, fmaxf(sr[kStageKeys - 2], sr[kStageKeys - 1])) * p.scale_log2;
         const float m_new = fmaxf(m_used, mx);
         const bool need = (m_new != -INFINITY) && (m_new > m_used + 8.0f);
         float alpha = 1.f;
@@ -655,22 +770,48 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
           m_used = m_new;
         }
         const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
-        const float sc = p.scale_log2;
-        // p = 2^(s*scale - m): packed FMA, then ex2; fp32 row sum before the bf16 rounding
+        if (KV8) {
+          // per half: p' = 2^(s * scale * sK - m + log2 sV) = sV * p, packed as f16
+          // for the f16 PV; the row sum takes sum(p') / sV = sum(p)
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-        for (int c = 0; c < kStageKeys / 32; ++c) {
-          if (c * 32 < nvalid) {
-            uint32_t pk[16];
+          for (int c = 0; c < kStageKeys / 32; ++c) {
+            if (c * 32 < nvalid) {
+              const float sc = c < 2 ? scA : scB;
+              const float bias = (c < 2 ? lbA : lbB) + nm;
+              uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float x0, x1;
-              ffma2(x0, x1, sr[c * 32 + 2 * i], sr[c * 32 + 2 * i + 1], sc, sc, nm, nm);
-              const float e0 = ex2(x0), e1 = ex2(x1);
-              if (i & 1) fadd2(l2, l3, e0, e1);  // two independent sum chains
-              else fadd2(l0, l1, e0, e1);
-              pk[i] = pack_bf16x2(e0, e1);
+              for (int i = 0; i < 16; ++i) {
+                float x0, x1;
+                ffma2(x0, x1, sr[c * 32 + 2 * i], sr[c * 32 + 2 * i + 1], sc, sc, bias, bias);
+                const float e0 = ex2(x0), e1 = ex2(x1);
+                if (c < 2) fadd2(a0, a1, e0, e1);
+                else fadd2(a2, a3, e0, e1);
+                pk[i] = pack_f16x2(e0, e1);
+              }
+              tmem_st16(tS + c * 16, pk);
             }
-            tmem_st16(tS + c * 16, pk);
+          }
+          l0 += (a0 + a1) * __frcp_rn(scl_a.y);
+          l2 += (a2 + a3) * __frcp_rn(scl_b.y);
+        } else {
+          const float sc = p.scale_log2;
+          // p = 2^(s*scale - m): packed FMA, then ex2; fp32 row sum before the bf16 rounding
+#pragma unroll
+          for (int c = 0; c < kStageKeys / 32; ++c) {
+            if (c * 32 < nvalid) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                float x0, x1;
+                ffma2(x0, x1, sr[c * 32 + 2 * i], sr[c * 32 + 2 * i + 1], sc, sc, nm, nm);
+                const float e0 = ex2(x0), e1 = ex2(x1);
+                if (i & 1) fadd2(l2, l3, e0, e1);  // two independent sum chains
+                else fadd2(l0, l1, e0, e1);
+                pk[i] = pack_bf16x2(e0, e1);
+              }
+              tmem_st16(tS + c * 16, pk);
+            }
           }
         }
         // O still holds the sum over earlier stages at the old max: bring it to the new one
@@ -943,6 +1084,41 @@ __global__ void __launch_bounds__(1024)
   if (tid == 0) *n_units = carry;
 }
 
+// bf16 -> f16 (exact for |x| in [2^-14, 65504]; smaller values round as f16
+// subnormals), for Q of the E4M3 path.
+__global__ void cast_bf16_f16_kernel(const __nv_bfloat16* __restrict__ src,
+                                     __half* __restrict__ dst, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    dst[i] = __float2half_rn(__bfloat162float(src[i]));
+}
+
+// escale[g * nKblk + e] = (K_scale, V_scale) of the page behind table entry e
+// of group g (entries past counts[g] are left as they are).
+__global__ void gather_scales_kernel(const int32_t* __restrict__ tables,
+                                     const int32_t* __restrict__ counts,
+                                     const int32_t* __restrict__ page_table,
+                                     const float* __restrict__ K_scale,
+                                     const float* __restrict__ V_scale, int Hkv, int nKblk,
+                                     int num_pages, float2* __restrict__ escale, int32_t* err) {
+  const int g = blockIdx.y;
+  const int cnt = min(max(counts[g], 0), nKblk);
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < cnt; e += gridDim.x * blockDim.x) {
+    int kb = tables[(size_t)g * nKblk + e];
+    if (kb < 0 || kb >= nKblk) {
+      set_flag(err, CA_FLAG_BOUNDS);
+      kb = 0;
+    }
+    int pg = page_table[kb];
+    if (pg < 0 || pg >= num_pages) {
+      set_flag(err, CA_FLAG_BOUNDS);
+      pg = 0;
+    }
+    escale[(size_t)g * nKblk + e] = make_float2(K_scale[(size_t)pg * Hkv + g],
+                                                V_scale[(size_t)pg * Hkv + g]);
+  }
+}
+
 // One CTA waits on a barrier nobody arrives on, for at most limit_ns.
 __global__ void wait_probe_kernel(int32_t* err, unsigned long long limit_ns) {
   __shared__ __align__(8) uint64_t bar;
@@ -959,34 +1135,38 @@ __global__ void wait_probe_kernel(int32_t* err, unsigned long long limit_ns) {
 
 namespace ca {
 
-template <int D, int NT, bool QS>
+template <int D, int NT, bool QS, bool KV8>
 static cudaError_t launch_attn_t(const CUtensorMap& q, const CUtensorMap& qlo,
                                  const CUtensorMap& k, const CUtensorMap& v, const AttnParams& p,
                                  int grid, cudaStream_t st) {
-  using S = Smem<D, NT, QS>;
+  using S = Smem<D, NT, QS, KV8>;
   static_assert(S::kAlloc <= 227 * 1024, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(chunk_attn_kernel<D, NT, QS>,
+  cudaError_t e = cudaFuncSetAttribute(chunk_attn_kernel<D, NT, QS, KV8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc);
   if (e != cudaSuccess) return e;
-  chunk_attn_kernel<D, NT, QS><<<grid, 128 + NT * 128, S::kAlloc, st>>>(q, qlo, k, v, p);
+  chunk_attn_kernel<D, NT, QS, KV8><<<grid, 128 + NT * 128, S::kAlloc, st>>>(q, qlo, k, v, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_chunk_attention(const CUtensorMap& q, const CUtensorMap& qlo,
                                    const CUtensorMap& k, const CUtensorMap& v,
-                                   const AttnParams& p, int D, int NT, bool qsplit, int grid,
-                                   cudaStream_t st) {
-#define CA_LAUNCH(d_, nt_, qs_)                                                  \
-  if (D == d_ && NT == nt_ && qsplit == qs_)                                     \
-    return launch_attn_t<d_, nt_, qs_>(q, qlo, k, v, p, grid, st);
-  CA_LAUNCH(128, 2, false)
-  CA_LAUNCH(128, 1, false)
-  CA_LAUNCH(64, 2, false)
-  CA_LAUNCH(64, 1, false)
-  CA_LAUNCH(128, 2, true)
-  CA_LAUNCH(128, 1, true)
-  CA_LAUNCH(64, 2, true)
-  CA_LAUNCH(64, 1, true)
+                                   const AttnParams& p, int D, int NT, bool qsplit, bool kv8,
+                                   int grid, cudaStream_t st) {
+#define CA_LAUNCH(d_, nt_, qs_, kv8_)                                            \
+  if (D == d_ && NT == nt_ && qsplit == qs_ && kv8 == kv8_)                      \
+    return launch_attn_t<d_, nt_, qs_, kv8_>(q, qlo, k, v, p, grid, st);
+  CA_LAUNCH(128, 2, false, false)
+  CA_LAUNCH(128, 1, false, false)
+  CA_LAUNCH(64, 2, false, false)
+  CA_LAUNCH(64, 1, false, false)
+  CA_LAUNCH(128, 2, true, false)
+  CA_LAUNCH(128, 1, true, false)
+  CA_LAUNCH(64, 2, true, false)
+  CA_LAUNCH(64, 1, true, false)
+  CA_LAUNCH(128, 2, false, true)
+  CA_LAUNCH(128, 1, false, true)
+  CA_LAUNCH(64, 2, false, true)
+  CA_LAUNCH(64, 1, false, true)
 #undef CA_LAUNCH
   return cudaErrorInvalidValue;
 }
@@ -1040,6 +1220,25 @@ cudaError_t launch_varlen_setup(const int32_t* cu_q, const int32_t* prefix_len,
                                 cudaStream_t st) {
   varlen_setup_kernel<<<1, 1024, 0, st>>>(cu_q, prefix_len, cu_pages, num_seqs, total_q, B, Hkv,
                                           nhalves, out, n_units, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cast_bf16_f16(const void* src, void* dst, size_t n, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  size_t blocks = (n + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  cast_bf16_f16_kernel<<<(unsigned)blocks, 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(src), static_cast<__half*>(dst), n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_scales(const int32_t* tables, const int32_t* counts,
+                                 const int32_t* page_table, const float* K_scale,
+                                 const float* V_scale, int Hkv, int nKblk, int num_pages,
+                                 float2* escale, int32_t* err, cudaStream_t st) {
+  const dim3 grid((nKblk + 255) / 256, Hkv);
+  gather_scales_kernel<<<grid, 256, 0, st>>>(tables, counts, page_table, K_scale, V_scale, Hkv,
+                                             nKblk, num_pages, escale, err);
   return cudaGetLastError();
 }
 

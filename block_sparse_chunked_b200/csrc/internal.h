@@ -46,6 +46,9 @@ struct AttnParams {
   int mask_words, nQblk_mask;
   int32_t* tables_out;
   int32_t* counts_out;
+  // E4M3 pages: per table entry (group g, entry e) the (K, V) scales of its
+  // page, escale[g * nKblk + e] (built by a gather kernel before the launch)
+  const float2* escale;
   const SeqDesc* seqs;  // [num_seqs] in device memory, or null: one sequence, seq0
   SeqDesc seq0;
   int num_seqs;
@@ -61,8 +64,13 @@ cudaError_t launch_build_tables_bits(const uint32_t* bits, int nb, int Hq, int H
                                      cudaStream_t stream);
 cudaError_t launch_chunk_attention(const CUtensorMap& q, const CUtensorMap& qlo,
                                    const CUtensorMap& k, const CUtensorMap& v,
-                                   const AttnParams& p, int D, int NT, bool qsplit, int grid,
-                                   cudaStream_t st);
+                                   const AttnParams& p, int D, int NT, bool qsplit, bool kv8,
+                                   int grid, cudaStream_t st);
+cudaError_t launch_cast_bf16_f16(const void* src, void* dst, size_t n, cudaStream_t st);
+cudaError_t launch_gather_scales(const int32_t* tables, const int32_t* counts,
+                                 const int32_t* page_table, const float* K_scale,
+                                 const float* V_scale, int Hkv, int nKblk, int num_pages,
+                                 float2* escale, int32_t* err, cudaStream_t st);
 cudaError_t launch_sk_combine(const AttnParams& p, int D, int NT, cudaStream_t st);
 cudaError_t launch_split_combine(const float* Opart, const float* LSEpart, int n_splits, int L,
                                  int Hq, int D, void* O, float* LSE, int out_f32,

@@ -53,6 +53,7 @@ extern "C" {
 
 #define CA_DTYPE_BF16 0
 #define CA_DTYPE_FP32 1
+#define CA_DTYPE_E4M3 2  /* K/V pages of ca_chunk_attention_fp8 (not a Q dtype) */
 
 /*
  * ca_build_tables — Q-block union + intra-group union + compaction
@@ -226,6 +227,41 @@ int ca_chunk_attention_masked(const void* Q, const void* K_pages, const void* V_
                               int prefix_len, int32_t* tables_out, int32_t* counts_out, void* O,
                               float* LSE, void* workspace, size_t ws_bytes, int n_splits,
                               int32_t* err_flag, void* stream);
+
+/*
+ * ca_chunk_attention_fp8 — ca_chunk_attention over an FP8 (E4M3) paged KV
+ * cache: half the bytes of a bf16 cache per token ("CompactAttention ...",
+ * Abstract: selected blocks read in place from the paged cache; the format
+ * of the cache is this library's choice).
+ *
+ * Page format: K_pages / V_pages hold one E4M3 byte per element (1 sign, 4
+ * exponent bits with bias 7, 3 mantissa bits; exponent 0 = subnormals; 0x7F
+ * / 0xFF are NaN), [num_pages, Hkv, B, d]; K_scale / V_scale float32
+ * [num_pages, Hkv] hold one positive, finite scale per (page, KV head):
+ * element = decode(byte) * scale.  The result is the single-sequence
+ * definition above evaluated on those decoded values.
+ *
+ * How: the bytes are staged by TMA and widened to f16 (exactly) in shared
+ * memory; Q is converted to f16 in the workspace (exact for |Q| in
+ * [2^-14, 65504], |Q| must stay below 65504); the MMAs run in f16 with fp32
+ * accumulation; the K scale multiplies the scores and the V scale the
+ * softmax weights inside the softmax, in fp32 (P is stored as f16, so the
+ * per-page scales of one sequence should stay within about 2^10 of each
+ * other).
+ *   Q       bf16 [L, Hq, d];  O bf16 [L, Hq, d];  LSE float32 [Hq, L]
+ *   workspace >= ca_workspace_size_fp8(...) bytes (never 0)
+ *   n_splits  <= 0 automatic (KV splits when the units do not fill the SMs),
+ *             k >= 1 as for ca_chunk_attention (no persistent grid)
+ * Limits: as ca_chunk_attention; one sequence per call.
+ */
+size_t ca_workspace_size_fp8(int Hq, int Hkv, int head_dim, int block, int chunk_len,
+                             int prefix_len, int num_pages, int n_splits);
+int ca_chunk_attention_fp8(const void* Q, const uint8_t* K_pages, const uint8_t* V_pages,
+                           const float* K_scale, const float* V_scale, int num_pages,
+                           const int32_t* page_table, const int32_t* tables,
+                           const int32_t* counts, int Hq, int Hkv, int head_dim, int block,
+                           int chunk_len, int prefix_len, void* O, float* LSE, void* workspace,
+                           size_t ws_bytes, int n_splits, int32_t* err_flag, void* stream);
 
 /*
  * ca_chunk_attention_noalloc — ca_chunk_attention (bf16 inputs) for callers

@@ -32,3 +32,9 @@ from .attention import (  # noqa: F401
     oracle_append_kv,
     oracle_varlen,
 )
+from .fp8 import (  # noqa: F401,E402
+    decode_e4m3,
+    dequantize_pages,
+    oracle_chunk_attention_fp8,
+    oracle_rows_fp8,
+)

@@ -191,3 +191,18 @@ def test_workspace_size_masked(bsc):
     assert wm(0, 32, 8, 128, 64, 2048, 129024, 2048, 0) == 0           # 256 units: one CTA each
     assert wm(0, 8, 2, 128, 64, 512, 1024, 24, 0) > 0                  # 16 units: KV splits
     assert wm(0, 32, 8, 128, 64, 2048, 129024 + 64, 2049, 0) == ctypes.c_size_t(-1).value
+
+
+def test_fp8_entry_rejects_bad_arguments(bsc):
+    f = bsc.lib.ca_chunk_attention_fp8
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, 40, FAKE, FAKE, FAKE, 8, 2, 128, 64, 256, 1024, FAKE,
+            FAKE, None, 0, 1, None, None]
+    assert f(*args) == bsc.CA_ERR_WORKSPACE          # the fp8 path always needs workspace
+    bad = list(args)
+    bad[3] = None                                    # no K scales
+    assert f(*bad) == bsc.CA_ERR_ARG
+    bad = list(args)
+    bad[11] = 96                                     # head_dim
+    assert f(*bad) == bsc.CA_ERR_ARG
+    assert bsc.lib.ca_workspace_size_fp8(8, 2, 128, 64, 256, 1024, 40, 1) > 0
+    assert bsc.lib.ca_workspace_size_fp8(8, 2, 128, 64, 256, 1024, 10, 1) == ctypes.c_size_t(-1).value

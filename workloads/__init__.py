@@ -15,4 +15,5 @@ from .generators import (  # noqa: F401
     mask_for,
     causal_live,
     last_live_block,
+    quantize_pages_e4m3,
 )

@@ -128,3 +128,18 @@ def pack_mask_bits(mask):
     pad = np.zeros(m.shape[:-1] + (W * 32 - nK,), dtype=bool)
     b = np.packbits(np.concatenate([m, pad], axis=-1), axis=-1, bitorder="little")
     return np.ascontiguousarray(b).view("<u4").astype(np.uint32)
+
+
+def quantize_pages_e4m3(pages, scale_factor=None):
+    """float pages [num_pages, Hkv, B, d] (torch) -> (uint8 E4M3 codes, float32 scales
+    [num_pages, Hkv]): one scale per (page, KV head) tile, amax / 448 (448 being the
+    largest E4M3 value) times an optional factor >= 1 per tile (coarser codes, so
+    that scales differ more between pages), codes by torch's round-to-nearest cast.
+    Input generation only: the decode belongs to each side."""
+    x = pages.float()
+    amax = x.abs().amax(dim=(2, 3))
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    if scale_factor is not None:
+        scale = scale * scale_factor
+    codes = (x / scale[:, :, None, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), scale.contiguous()
