@@ -34,7 +34,6 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
-#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -57,8 +56,8 @@ __device__ __forceinline__ void set_flag(int32_t* err, int f) {
 // S = Q_hi K^T + Q_lo K^T, which removes the rounding error of Q (the error
 // term shared by all keys of a row); used for fp32 inputs.
 //
-// KV8: K/V pages hold E4M3 bytes; TMA brings a stage's K and V bytes into a
-// staging area, warps 2-3 widen them to f16 into the swizzled operand ring, and
+// KV8: K/V pages hold E4M3 bytes; TMA brings a stage's K and V bytes into two
+// staging halves, warps 2-3 widen them to f16 into the swizzled operand ring, and
 // the MMAs run kind::f16 with f16 operands (Q converted to f16, P written as
 // f16).  The per-page scales are applied in the softmax.
 template <int D, int NT, bool QSPLIT, bool KV8 = false>
@@ -77,8 +76,9 @@ struct Smem {
   static constexpr int kStgOff = kVOff + kNS * kKV;
   static constexpr int kBarOff = kStgOff + kStg;
   // barriers: q_full, full_k[NS], full_v[NS], empty_k[NS], empty_v[NS],
-  //           s_full[2], p_full[2], o_done, drain, q_free (+ stg_full, stg_empty)
-  static constexpr int kNumBars = 1 + 4 * kNS + 2 + 2 + 3 + (KV8 ? 2 : 0);
+  //           s_full[2], p_full[2], o_done, drain, q_free
+  //           (+ KV8: stg_full[2], stg_empty[2] for the K and V staging halves)
+  static constexpr int kNumBars = 1 + 4 * kNS + 2 + 2 + 3 + (KV8 ? 4 : 0);
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   // persistent schedule: per-unit live entries, prefix of stage counts, warp sums
   // (not used with E4M3 pages, which run one CTA per unit or KV splits)
@@ -254,8 +254,9 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
   const uint32_t o_done = bars + 8u * (5 + 4 * kNS);
   const uint32_t drain = bars + 8u * (6 + 4 * kNS);
   const uint32_t q_free = bars + 8u * (7 + 4 * kNS);
-  const uint32_t stg_full = bars + 8u * (8 + 4 * kNS);   // KV8 only
-  const uint32_t stg_empty = bars + 8u * (9 + 4 * kNS);  // KV8 only
+  // KV8 only: staging half h (0 = K, 1 = V) loaded / widened
+  auto stg_full = [&](int h) { return bars + 8u * (8 + 4 * kNS + h); };
+  auto stg_empty = [&](int h) { return bars + 8u * (10 + 4 * kNS + h); };
   int* misc = reinterpret_cast<int*>(sm + S::kMiscOff);
   // misc[0] tmem base, [1] live entries (one-piece mode), [2] first stage,
   // [3] last stage (exclusive), [4] live entries of the fused table (thread 0
@@ -353,8 +354,10 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
     if (KV8) {
-      mbar_init(stg_full, 1);
-      mbar_init(stg_empty, 2);
+      for (int h = 0; h < 2; ++h) {
+        mbar_init(stg_full(h), 1);
+        mbar_init(stg_empty(h), 2);
+      }
     }
     fence_mbar_init();
   }
@@ -464,18 +467,17 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
           page[pi] = __shfl_sync(0xffffffffu, pg_cache, e - cache_base);
         }
         if (KV8) {
-          // E4M3 bytes of the stage's pages into the staging area, once the
-          // widening warps have finished with the previous stage's bytes
-          if (gj > 0) ok = wait_warp(stg_empty, (gj - 1) & 1, p, abort_flag);
-          if (ok) {
-            const uint32_t b8 = (uint32_t)npg * p.B * D;
-            mbar_expect_tx_w(stg_full, 2 * b8);
+          // E4M3 bytes of the stage's pages into the staging halves (K, then
+          // V), each as soon as the widening warps are done with its previous
+          // contents, so one half loads while the other is widened
+          const uint32_t b8 = (uint32_t)npg * p.B * D;
+          for (int h = 0; h < 2 && ok; ++h) {
+            if (gj > 0) ok = wait_warp(stg_empty(h), (gj - 1) & 1, p, abort_flag);
+            if (!ok) break;
+            mbar_expect_tx_w(stg_full(h), b8);
             for (int pi = 0; pi < npg; ++pi)
-              tma_load_4d_w(sbase + S::kStgOff + pi * p.B * D, &tmK, stg_full, 0, 0, uc.g,
-                            page[pi], pol);
-            for (int pi = 0; pi < npg; ++pi)
-              tma_load_4d_w(sbase + S::kStgOff + kStageKeys * D + pi * p.B * D, &tmV, stg_full,
-                            0, 0, uc.g, page[pi], pol);
+              tma_load_4d_w(sbase + S::kStgOff + h * kStageKeys * D + pi * p.B * D,
+                            h ? &tmV : &tmK, stg_full(h), 0, 0, uc.g, page[pi], pol);
           }
           continue;
         }
@@ -501,7 +503,10 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
     if (lane == 0) {
       // Do not leave with copies in flight: the last stages' loads must land.
       if (KV8) {
-        if (gj > 0) mbar_wait(stg_full, (gj - 1) & 1, p.wait_ns);
+        if (gj > 0) {
+          mbar_wait(stg_full(0), (gj - 1) & 1, p.wait_ns);
+          mbar_wait(stg_full(1), (gj - 1) & 1, p.wait_ns);
+        }
       } else {
         for (int G = max(0, gj - kNS); G < gj; ++G) {
           mbar_wait(full_k(G % kNS), (G / kNS) & 1, p.wait_ns);
@@ -627,13 +632,17 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
         const int r = i / CPR, q = i % CPR;
         const uint4 x = *reinterpret_cast<const uint4*>(src + r * D + q * 16);
         const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        // E4M3 byte b -> f16 bits (sign << 15) | ((b & 0x7F) << 7): that f16 is
+        // decode(b) / 256 for every non-NaN code, subnormals included (the f16
+        // exponent bias is 8 above E4M3's and E4M3 subnormals land on f16
+        // subnormals); the 256 is folded into the page scales.  Integer ops
+        // only, leaving the SFU / conversion pipe to the exponentials.
         uint32_t h[8];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] & 0xffffu), __NV_E4M3);
-          const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] >> 16), __NV_E4M3);
-          h[2 * k] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
-          h[2 * k + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
+          const uint32_t t0 = __byte_perm(w[k], 0u, 0x4140), t1 = __byte_perm(w[k], 0u, 0x4342);
+          h[2 * k] = ((t0 & 0x00800080u) << 8) | ((t0 & 0x007F007Fu) << 7);
+          h[2 * k + 1] = ((t1 & 0x00800080u) << 8) | ((t1 & 0x007F007Fu) << 7);
         }
         const int u = (q & 3) * 2;  // first 16-byte unit of these 16 elements in their row
         uint8_t* rowp = dst + (q >> 2) * S::kChunkBytes + r * 128;
@@ -648,17 +657,21 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
       for (int stage = s0; stage < s1 && ok; ++stage, ++gj) {
         const int slot = gj % kNS, round = gj / kNS;
         const int rows = min(spb, live - stage * spb) * p.B;
-        ok = wait_warp(stg_full, gj & 1, p, abort_flag);
+        ok = wait_warp(stg_full(0), gj & 1, p, abort_flag);
         if (ok && round > 0) ok = wait_warp(empty_k(slot), (round - 1) & 1, p, abort_flag);
         if (!ok) break;
         widen(S::kStgOff, S::kKOff + slot * S::kKV, rows);
-        if (lane == 0) mbar_arrive(full_k(slot));
-        if (round > 0) ok = wait_warp(empty_v(slot), (round - 1) & 1, p, abort_flag);
+        if (lane == 0) {
+          mbar_arrive(full_k(slot));
+          mbar_arrive(stg_empty(0));
+        }
+        ok = wait_warp(stg_full(1), gj & 1, p, abort_flag);
+        if (ok && round > 0) ok = wait_warp(empty_v(slot), (round - 1) & 1, p, abort_flag);
         if (!ok) break;
         widen(S::kStgOff + kStageKeys * D, S::kVOff + slot * S::kKV, rows);
         if (lane == 0) {
           mbar_arrive(full_v(slot));
-          mbar_arrive(stg_empty);
+          mbar_arrive(stg_empty(1));
         }
       }
     });
@@ -1093,8 +1106,8 @@ __global__ void cast_bf16_f16_kernel(const __nv_bfloat16* __restrict__ src,
     dst[i] = __float2half_rn(__bfloat162float(src[i]));
 }
 
-// escale[g * nKblk + e] = (K_scale, V_scale) of the page behind table entry e
-// of group g (entries past counts[g] are left as they are).
+// escale[g * nKblk + e] = 256 * (K_scale, V_scale) of the page behind table
+// entry e of group g (entries past counts[g] are left as they are).
 __global__ void gather_scales_kernel(const int32_t* __restrict__ tables,
                                      const int32_t* __restrict__ counts,
                                      const int32_t* __restrict__ page_table,
@@ -1114,8 +1127,9 @@ __global__ void gather_scales_kernel(const int32_t* __restrict__ tables,
       set_flag(err, CA_FLAG_BOUNDS);
       pg = 0;
     }
-    escale[(size_t)g * nKblk + e] = make_float2(K_scale[(size_t)pg * Hkv + g],
-                                                V_scale[(size_t)pg * Hkv + g]);
+    // x 256: the widened f16 operands hold decode(byte) / 256
+    escale[(size_t)g * nKblk + e] = make_float2(K_scale[(size_t)pg * Hkv + g] * 256.f,
+                                                V_scale[(size_t)pg * Hkv + g] * 256.f);
   }
 }
 
