@@ -10,9 +10,10 @@
 // The unit's rows are the span's 64 tokens for up to four query heads of the
 // group, stacked into NT = 1 or 2 tensor-core tiles of 128 rows (two heads per
 // tile).  All rows of a unit share the group's table, so every KV block
-// fetched from HBM/L2 feeds 2*NT MMAs.  Because the chunk starts on a block
-// boundary, the blocks a span may see are a prefix of the sorted table
-// (entries <= the span's diagonal block), and only the diagonal block needs a
+// fetched from HBM/L2 feeds 2*NT MMAs.  The blocks a span may see are a prefix
+// of the sorted table (entries whose block holds a position <= the span's last
+// query), and only the last one or two of them (those past the span's first
+// query position: for a block-aligned chunk, the diagonal block) need a
 // token-level causal mask.
 //
 // One CTA per unit (1 CTA / SM: it holds all 512 TMEM columns):
