@@ -199,6 +199,8 @@ cudaError_t launch_build_tables(const uint8_t* mask, int nb, int Hq, int Hkv, in
   C = C > 8 ? 8 : C;
   const int cmax = (nKblk + 255) / 256;
   C = C > cmax ? cmax : C;
+  const int cmin = (nKblk + kMaxSlab - 1) / kMaxSlab;  // slabs of at most kMaxSlab columns
+  if (C < cmin) C = cmin;                              // (<= 8 for nKblk <= 65536)
   if (C < 1) C = 1;
   int slab = (nKblk + C - 1) / C;
   slab = (slab + 31) & ~31;

@@ -119,3 +119,24 @@ def test_repeatable_and_overwrites_stale_output(bsc):
     assert torch.equal(t, t1) and torch.equal(c, c1)
     to, co = oracle.oracle_tables(workloads.mask_for(w), w.Hkv)
     assert np.array_equal(t.cpu().numpy(), to)
+
+
+@pytest.mark.parametrize("nb,Hq,Hkv,nQ,nK,rho", [
+    (16, 32, 8, 32, 2048, None),      # 128 (mask, group) units of the 128K config
+    (40, 8, 4, 3, 1000, 0.05),        # ragged width: 4-byte loads
+    (130, 4, 1, 2, 37, 0.3),          # odd width: 1-byte loads
+    (32, 8, 4, 2, 20000, 0.01),       # many units and a wide table: 3 slabs per cluster
+    (64, 2, 2, 1, 33000, 0.001),      # wider than 4 slabs: the cluster grows to 5
+])
+def test_batched_many_masks_and_wide_tables(bsc, nb, Hq, Hkv, nQ, nK, rho):
+    if rho is None:
+        w = workloads.get_config("ctx128k")
+        masks = np.stack([workloads.mask_for(w, seed=s) for s in range(nb)])
+    else:
+        rng = np.random.default_rng(nb + nK)
+        masks = (rng.random((nb, Hq, nQ, nK)) < rho).astype(np.uint8)
+    t, c = bsc.build_tables_batched(torch.from_numpy(masks).cuda(), Hkv)
+    t, c = t.cpu().numpy(), c.cpu().numpy()
+    for s in range(nb):
+        to, co = oracle.oracle_tables(masks[s], Hkv)
+        assert np.array_equal(t[s], to) and np.array_equal(c[s], co), s
