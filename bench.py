@@ -216,6 +216,61 @@ def run_sweep(bsc, dev, stream, n_chunks=32):
             "per_chunk_ms_first_last": [method_ms[0], method_ms[-1]]}
 
 
+def run_varlen(bsc, dev, stream, reps=12):
+    """A batch of 8 sequences with unaligned prefixes and chunk lengths over one
+    shuffled page pool, through one ca_chunk_attention_varlen launch (tables
+    built per sequence beforehand).  Seeded device data; 32/8 heads, d 128."""
+    import numpy as np
+    import torch
+
+    import workloads as wl
+    seqs = [(121037, 2048), (64005, 1500), (32868, 1024), (100063, 777), (8000, 512),
+            (120001, 2000), (50030, 1900), (90011, 1100)]
+    Hq, Hkv, d, B = 32, 8, 128, 64
+    nKs = [-(-(P + L) // B) for P, L in seqs]
+    num_pages = sum(nKs)
+    g = torch.Generator(device=dev).manual_seed(0)
+    K = torch.randn(num_pages, Hkv, B, d, generator=g, device=dev).bfloat16()
+    V = torch.randn(num_pages, Hkv, B, d, generator=g, device=dev).bfloat16()
+    rng = np.random.default_rng(0)
+    pt = torch.from_numpy(rng.permutation(num_pages).astype(np.int32)).to(dev)
+    cu_q = torch.tensor(np.concatenate([[0], np.cumsum([L for _, L in seqs])]), dtype=torch.int32,
+                        device=dev)
+    cu_pages = torch.tensor(np.concatenate([[0], np.cumsum(nKs)]), dtype=torch.int32, device=dev)
+    prefix = torch.tensor([P for P, _ in seqs], dtype=torch.int32, device=dev)
+    total_q = int(cu_q[-1])
+    Q = torch.randn(total_q, Hq, d, generator=g, device=dev).bfloat16()
+    flat = torch.full((Hkv * num_pages,), -1, dtype=torch.int32, device=dev)
+    counts = torch.zeros(len(seqs), Hkv, dtype=torch.int32, device=dev)
+    flops = 0.0
+    off = 0
+    for s, (P, L) in enumerate(seqs):
+        w = wl.Workload("vb", Hq, Hkv, d, "bf16", P, L, B, "vslash", rho=0.05, corr=0.7,
+                        window=8, seed=s)
+        t = flat[Hkv * off:Hkv * (off + nKs[s])].view(Hkv, nKs[s])
+        bsc.build_tables(torch.from_numpy(wl.mask_for(w)).to(dev), Hkv, t, counts[s])
+        flops += bsc.selected_flops_pl(t.cpu().numpy(), counts[s].cpu().numpy(), Hq, P, L, B, d)
+        off += nKs[s]
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    O = torch.empty_like(Q)
+    lse = torch.empty(Hq, total_q, dtype=torch.float32, device=dev)
+    max_kv = max(P + L for P, L in seqs)
+    n = bsc.lib.ca_workspace_size_varlen(0, Hq, Hkv, d, B, len(seqs), total_q, max_kv, num_pages, 1)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    ts = []
+    for r in range(reps):
+        t_ = timed_launch(stream, lambda: bsc.chunk_attention_varlen(
+            Q, K, V, cu_q, prefix, pt, cu_pages, flat, counts, max_kv, n_splits=1, err_flag=err,
+            out=O, lse=lse, workspace=ws))
+        if r >= 3:
+            ts.append(t_)
+    bsc.check(err)
+    ms = sum(ts) / len(ts)
+    return {"sequences": len(seqs), "query_tokens": total_q, "kv_tokens": sum(P + L for P, L in seqs),
+            "ms": ms, "selected_gflop": flops / 1e9, "tflops": flops / (ms * 1e-3) / 1e12,
+            "note": "ca_chunk_attention_varlen, unaligned prefixes and chunk lengths, one launch"}
+
+
 def timed_launch(stream, fn):
     """Device time (ms) of the launches fn() makes.  A sleep kernel keeps the
     GPU busy while the host enqueues them, so the host-side call overhead of a
@@ -521,6 +576,9 @@ def main():
                        "buffer (not rotated)"}
     del K8, V8
 
+    # ---- a batch of sequences with unaligned lengths (one varlen launch)
+    varlen_res = run_varlen(bsc, dev, stream)
+
     # ---- the full chunked-prefill sweep (32 x 4096 tokens), one pass
     sweep_res = run_sweep(bsc, dev, stream)
 
@@ -637,6 +695,7 @@ def main():
             "sweep_131k": sweep_res,
             "fused_step": fused_res,
             "fp8_kv": fp8_res,
+            "varlen_batch": varlen_res,
             "kv_append": append_res,
             "table_build_batched": {"masks_per_launch": nb, "us": statistics.mean(bt) * 1e3,
                                     "GB/s": build_gbs, "frac_of_measured_hbm": build_gbs / hbm,

@@ -34,4 +34,11 @@ from ._capi import (  # noqa: F401
     wait_probe,
     last_error,
 )
-from .accounting import selected_pairs, selected_flops, dense_flops, builder_bytes  # noqa: F401
+from .accounting import (  # noqa: F401
+    selected_pairs,
+    selected_flops,
+    selected_pairs_pl,
+    selected_flops_pl,
+    dense_flops,
+    builder_bytes,
+)

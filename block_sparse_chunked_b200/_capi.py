@@ -112,6 +112,38 @@ def _need_cuda(name, t, dtypes=None, ndim=None):
         raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
 
 
+def _out(name, t, like_device, dtype, numel):
+    """A caller-provided output buffer: CUDA, contiguous, of the given dtype,
+    on the inputs' device and large enough (the kernels write numel elements)."""
+    _need_cuda(name, t, (dtype,))
+    if t.device != like_device:
+        raise ValueError(f"{name} is on {t.device}, the inputs on {like_device}")
+    if t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, {numel} needed")
+    return t
+
+
+def _errp(err_flag):
+    """Pointer to the caller's device error word (int32 CUDA tensor), or None."""
+    if err_flag is None:
+        return None
+    _need_cuda("err_flag", err_flag, (torch.int32,))
+    if err_flag.numel() < 1:
+        raise ValueError("err_flag must hold one int32")
+    return _ptr(err_flag)
+
+
+def _workspace(ws, nbytes, device):
+    """The caller's workspace if it is a contiguous CUDA tensor on `device` with at
+    least nbytes bytes, else a fresh uint8 buffer (None when nbytes is 0)."""
+    if nbytes == 0:
+        return None
+    if (ws is not None and isinstance(ws, torch.Tensor) and ws.is_cuda and ws.is_contiguous()
+            and ws.device == device and ws.numel() * ws.element_size() >= nbytes):
+        return ws
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
 def build_tables_batched(masks, Hkv, tables=None, counts=None):
     """masks uint8/bool [nb, Hq, nQblk, nKblk] -> tables int32 [nb, Hkv, nKblk], counts [nb, Hkv]."""
     _need_cuda("masks", masks, (torch.uint8, torch.bool), 4)
@@ -120,6 +152,8 @@ def build_tables_batched(masks, Hkv, tables=None, counts=None):
         tables = torch.empty(nb, Hkv, nK, dtype=torch.int32, device=masks.device)
     if counts is None:
         counts = torch.empty(nb, Hkv, dtype=torch.int32, device=masks.device)
+    _out("tables", tables, masks.device, torch.int32, nb * Hkv * nK)
+    _out("counts", counts, masks.device, torch.int32, nb * Hkv)
     _ok(lib.ca_build_tables_batched(_ptr(masks), nb, Hq, Hkv, nQ, nK, _ptr(tables), _ptr(counts),
                                     _stream()))
     return tables, counts
@@ -133,6 +167,8 @@ def build_tables(mask, Hkv, tables=None, counts=None):
         tables = torch.empty(Hkv, nK, dtype=torch.int32, device=mask.device)
     if counts is None:
         counts = torch.empty(Hkv, dtype=torch.int32, device=mask.device)
+    _out("tables", tables, mask.device, torch.int32, Hkv * nK)
+    _out("counts", counts, mask.device, torch.int32, Hkv)
     _ok(lib.ca_build_tables(_ptr(mask), Hq, Hkv, nQ, nK, _ptr(tables), _ptr(counts), _stream()))
     return tables, counts
 
@@ -148,6 +184,8 @@ def build_tables_bits(mask_bits, Hkv, nKblk, tables=None, counts=None):
         tables = torch.empty(nb, Hkv, nKblk, dtype=torch.int32, device=mask_bits.device)
     if counts is None:
         counts = torch.empty(nb, Hkv, dtype=torch.int32, device=mask_bits.device)
+    _out("tables", tables, mask_bits.device, torch.int32, nb * Hkv * nKblk)
+    _out("counts", counts, mask_bits.device, torch.int32, nb * Hkv)
     _ok(lib.ca_build_tables_bits(_ptr(mask_bits), nb, Hq, Hkv, nQ, nKblk, _ptr(tables),
                                  _ptr(counts), _stream()))
     return tables, counts
@@ -192,15 +230,16 @@ def chunk_attention(Q, K_pages, V_pages, page_table, tables, counts, prefix_len,
     code = _DT[Q.dtype]
     if out is None:
         out = torch.empty_like(Q)
+    _out("out", out, Q.device, Q.dtype, Q.numel())
     if lse is None:
         lse = torch.empty(Hq, L, dtype=torch.float32, device=Q.device)
+    _out("lse", lse, Q.device, torch.float32, Hq * L)
     ws_n = workspace_size(code, Hq, Hkv, d, B, L, prefix_len, num_pages, n_splits)
-    if ws_n and (workspace is None or workspace.numel() < ws_n):
-        workspace = torch.empty(ws_n, dtype=torch.uint8, device=Q.device)
+    workspace = _workspace(workspace, ws_n, Q.device)
     _ok(lib.ca_chunk_attention(
         _ptr(Q), _ptr(K_pages), _ptr(V_pages), code, num_pages, _ptr(page_table), _ptr(tables),
         _ptr(counts), Hq, Hkv, d, B, L, prefix_len, _ptr(out), _ptr(lse),
-        _ptr(workspace) if ws_n else None, ws_n, n_splits, _ptr(err_flag), _stream()))
+        _ptr(workspace) if ws_n else None, ws_n, n_splits, _errp(err_flag), _stream()))
     return out, lse
 
 
@@ -226,17 +265,18 @@ def chunk_attention_fp8(Q, K8, V8, K_scale, V_scale, page_table, tables, counts,
         raise ValueError("inconsistent shapes for chunk_attention_fp8")
     if out is None:
         out = torch.empty_like(Q)
+    _out("out", out, Q.device, Q.dtype, Q.numel())
     if lse is None:
         lse = torch.empty(Hq, L, dtype=torch.float32, device=Q.device)
+    _out("lse", lse, Q.device, torch.float32, Hq * L)
     ws_n = lib.ca_workspace_size_fp8(Hq, Hkv, d, B, L, prefix_len, num_pages, n_splits)
     if ws_n == ctypes.c_size_t(-1).value:
         raise CompactAttnError(CA_ERR_ARG, "invalid shapes for ca_workspace_size_fp8")
-    if workspace is None or workspace.numel() < ws_n:
-        workspace = torch.empty(ws_n, dtype=torch.uint8, device=Q.device)
+    workspace = _workspace(workspace, ws_n, Q.device)
     _ok(lib.ca_chunk_attention_fp8(
         _ptr(Q), _ptr(K8), _ptr(V8), _ptr(K_scale), _ptr(V_scale), num_pages, _ptr(page_table),
         _ptr(tables), _ptr(counts), Hq, Hkv, d, B, L, prefix_len, _ptr(out), _ptr(lse),
-        _ptr(workspace), ws_n, n_splits, _ptr(err_flag), _stream()))
+        _ptr(workspace), ws_n, n_splits, _errp(err_flag), _stream()))
     return out, lse
 
 
@@ -267,17 +307,18 @@ def chunk_attention_masked(Q, K_pages, V_pages, page_table, mask_bits, prefix_le
     code = _DT[Q.dtype]
     if out is None:
         out = torch.empty_like(Q)
+    _out("out", out, Q.device, Q.dtype, Q.numel())
     if lse is None:
         lse = torch.empty(Hq, L, dtype=torch.float32, device=Q.device)
+    _out("lse", lse, Q.device, torch.float32, Hq * L)
     ws_n = lib.ca_workspace_size_masked(code, Hq, Hkv, d, B, L, prefix_len, num_pages, n_splits)
     if ws_n == ctypes.c_size_t(-1).value:
         raise CompactAttnError(CA_ERR_ARG, "invalid shapes for ca_workspace_size_masked")
-    if ws_n and (workspace is None or workspace.numel() < ws_n):
-        workspace = torch.empty(ws_n, dtype=torch.uint8, device=Q.device)
+    workspace = _workspace(workspace, ws_n, Q.device)
     _ok(lib.ca_chunk_attention_masked(
         _ptr(Q), _ptr(K_pages), _ptr(V_pages), code, num_pages, _ptr(page_table), _ptr(mask_bits),
         Hq, Hkv, d, B, L, prefix_len, _ptr(tables_out), _ptr(counts_out), _ptr(out), _ptr(lse),
-        _ptr(workspace) if ws_n else None, ws_n, n_splits, _ptr(err_flag), _stream()))
+        _ptr(workspace) if ws_n else None, ws_n, n_splits, _errp(err_flag), _stream()))
     return out, lse
 
 
@@ -308,19 +349,20 @@ def chunk_attention_varlen(Q, K_pages, V_pages, cu_q, prefix_len, page_table, cu
     code = _DT[Q.dtype]
     if out is None:
         out = torch.empty_like(Q)
+    _out("out", out, Q.device, Q.dtype, Q.numel())
     if lse is None:
         lse = torch.empty(Hq, total_q, dtype=torch.float32, device=Q.device)
+    _out("lse", lse, Q.device, torch.float32, Hq * total_q)
     ws_n = lib.ca_workspace_size_varlen(code, Hq, Hkv, d, B, S, total_q, max_kv_len, num_pages,
                                         n_splits)
     if ws_n == ctypes.c_size_t(-1).value:
         raise CompactAttnError(CA_ERR_ARG, "invalid shapes for ca_workspace_size_varlen")
-    if workspace is None or workspace.numel() < ws_n:
-        workspace = torch.empty(ws_n, dtype=torch.uint8, device=Q.device)
+    workspace = _workspace(workspace, ws_n, Q.device)
     _ok(lib.ca_chunk_attention_varlen(
         _ptr(Q), _ptr(K_pages), _ptr(V_pages), code, num_pages, S, total_q, _ptr(cu_q),
         _ptr(prefix_len), max_kv_len, _ptr(page_table), _ptr(cu_pages), _ptr(tables),
         _ptr(counts), Hq, Hkv, d, B, _ptr(out), _ptr(lse), _ptr(workspace), ws_n, n_splits,
-        _ptr(err_flag), _stream()))
+        _errp(err_flag), _stream()))
     return out, lse
 
 
@@ -336,14 +378,14 @@ def append_kv(K_new, V_new, K_pages, V_pages, page_table, prefix_len, err_flag=N
     if V_new.shape != K_new.shape or V_pages.shape != K_pages.shape or Hkv2 != Hkv or d2 != d:
         raise ValueError("append_kv: inconsistent shapes")
     _ok(lib.ca_append_kv(_ptr(K_new), _ptr(V_new), _DT[K_new.dtype], _ptr(K_pages), _ptr(V_pages),
-                         num_pages, _ptr(page_table), Hkv, d, B, prefix_len, L, _ptr(err_flag),
+                         num_pages, _ptr(page_table), Hkv, d, B, prefix_len, L, _errp(err_flag),
                          _stream()))
 
 
 def check(err_flag):
     """Synchronise, read and clear the device error word; raise on a device error."""
-    _ok(lib.ca_check(_ptr(err_flag), _stream()))
+    _ok(lib.ca_check(_errp(err_flag), _stream()))
 
 
 def wait_probe(err_flag, limit_us):
-    _ok(lib.ca_wait_probe(_ptr(err_flag), int(limit_us), _stream()))
+    _ok(lib.ca_wait_probe(_errp(err_flag), int(limit_us), _stream()))

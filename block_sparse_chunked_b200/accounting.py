@@ -23,6 +23,27 @@ def selected_pairs(tables, counts, Hq, nPblk, nQblk):
     return total
 
 
+def selected_pairs_pl(tables, counts, Hq, P, L, B):
+    """selected_pairs for any prefix P and chunk length L: Q-block qb (chunk
+    tokens [qb B, min(qb B + B, L))) is live against the table entries up to
+    block (P + its last token) // B."""
+    tables = np.asarray(tables)
+    counts = np.asarray(counts)
+    Hkv = tables.shape[0]
+    G = Hq // Hkv
+    nQ = -(-L // B)
+    last = (P + np.minimum(np.arange(nQ) * B + B - 1, L - 1)) // B
+    total = 0
+    for g in range(Hkv):
+        row = np.sort(tables[g, :int(counts[g])])
+        total += G * int(np.searchsorted(row, last, side="right").sum())
+    return total
+
+
+def selected_flops_pl(tables, counts, Hq, P, L, B, head_dim):
+    return 4.0 * B * B * head_dim * selected_pairs_pl(tables, counts, Hq, P, L, B)
+
+
 def dense_pairs(Hq, nPblk, nQblk):
     return Hq * int(sum(nPblk + qb + 1 for qb in range(nQblk)))
 

@@ -206,3 +206,27 @@ def test_fp8_entry_rejects_bad_arguments(bsc):
     assert f(*bad) == bsc.CA_ERR_ARG
     assert bsc.lib.ca_workspace_size_fp8(8, 2, 128, 64, 256, 1024, 40, 1) > 0
     assert bsc.lib.ca_workspace_size_fp8(8, 2, 128, 64, 256, 1024, 10, 1) == ctypes.c_size_t(-1).value
+
+
+def test_accounting_general_lengths_match_aligned(bsc):
+    import numpy as np
+    import oracle
+    import workloads
+    w = workloads.get_config("llama16k")
+    t, c = oracle.oracle_tables(workloads.mask_for(w), w.Hkv)
+    a = bsc.selected_pairs(t, c, w.Hq, w.nPblk, w.nQblk)
+    b = bsc.selected_pairs_pl(t, c, w.Hq, w.prefix_len, w.chunk_len, w.block)
+    assert a == b
+    # unaligned: brute force over (h, qb, entry)
+    P, L, B, Hq, Hkv = 100, 70, 64, 4, 2
+    nK = -(-(P + L) // B)
+    rng = np.random.default_rng(0)
+    m = (rng.random((Hq, -(-L // B), nK)) < 0.5).astype(np.uint8)
+    t, c = oracle.oracle_tables(m, Hkv)
+    brute = 0
+    for h in range(Hq):
+        g = h // (Hq // Hkv)
+        for qb in range(-(-L // B)):
+            last_tok = min(qb * B + B - 1, L - 1)
+            brute += sum(1 for e in t[g, :c[g]] if e * B <= P + last_tok)
+    assert bsc.selected_pairs_pl(t, c, Hq, P, L, B) == brute
