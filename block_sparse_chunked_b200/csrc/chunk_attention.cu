@@ -625,31 +625,38 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
     const int ct = threadIdx.x - 64;  // 0 .. 63
     int gj = 0;
     bool ok = true;
+    // Thread ct always handles the same 16-byte column chunk q of rows r0,
+    // r0 + RS, ...; RS is a multiple of 8, so the row's swizzle phase (r & 7)
+    // and hence both 16-byte destination units are fixed per thread.
+    constexpr int CPR = D / 16;   // 16-byte chunks per E4M3 row
+    constexpr int RS = 64 / CPR;  // rows between a thread's chunks (8 or 16)
+    static_assert(RS % 8 == 0, "swizzle phase must repeat");
+    const int q = ct % CPR, r0 = ct / CPR;
+    const int u = (q & 3) * 2;  // first 16-byte unit of these 16 elements in a row
+    const uint32_t dst_lo = (q >> 2) * S::kChunkBytes + ((u ^ (r0 & 7)) << 4);
+    const uint32_t dst_hi = (q >> 2) * S::kChunkBytes + (((u + 1) ^ (r0 & 7)) << 4);
+    // E4M3 byte b -> f16 bits (sign << 15) | ((b & 0x7F) << 7): that f16 is
+    // decode(b) / 256 for every non-NaN code, subnormals included (the f16
+    // exponent bias is 8 above E4M3's and E4M3 subnormals land on f16
+    // subnormals); the 256 is folded into the page scales.  With a pair of bytes
+    // placed in the high byte of each 16-bit half (t), y = t >> 1 puts the
+    // magnitude at bits 7..13 and the sign at bit 14, and y + (y & 0x4000)
+    // moves the sign to bit 15.  Integer ops only, leaving the SFU to the
+    // exponentials.
+    auto pair = [](uint32_t w, uint32_t sel) {
+      const uint32_t y = __byte_perm(w, 0u, sel) >> 1;
+      return y + (y & 0x40004000u);
+    };
     auto widen = [&](uint32_t src_off, uint32_t dst_off, int rows) {
-      constexpr int CPR = D / 16;  // 16-byte chunks per E4M3 row
-      const uint8_t* src = sm + src_off;
+      const uint8_t* src = sm + src_off + q * 16;
       uint8_t* dst = sm + dst_off;
-      for (int i = ct; i < rows * CPR; i += 64) {
-        const int r = i / CPR, q = i % CPR;
-        const uint4 x = *reinterpret_cast<const uint4*>(src + r * D + q * 16);
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-        // E4M3 byte b -> f16 bits (sign << 15) | ((b & 0x7F) << 7): that f16 is
-        // decode(b) / 256 for every non-NaN code, subnormals included (the f16
-        // exponent bias is 8 above E4M3's and E4M3 subnormals land on f16
-        // subnormals); the 256 is folded into the page scales.  Integer ops
-        // only, leaving the SFU / conversion pipe to the exponentials.
-        uint32_t h[8];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t t0 = __byte_perm(w[k], 0u, 0x4140), t1 = __byte_perm(w[k], 0u, 0x4342);
-          h[2 * k] = ((t0 & 0x00800080u) << 8) | ((t0 & 0x007F007Fu) << 7);
-          h[2 * k + 1] = ((t1 & 0x00800080u) << 8) | ((t1 & 0x007F007Fu) << 7);
-        }
-        const int u = (q & 3) * 2;  // first 16-byte unit of these 16 elements in their row
-        uint8_t* rowp = dst + (q >> 2) * S::kChunkBytes + r * 128;
-        *reinterpret_cast<uint4*>(rowp + ((u ^ (r & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<uint4*>(rowp + (((u + 1) ^ (r & 7)) << 4)) =
-            make_uint4(h[4], h[5], h[6], h[7]);
+      for (int r = r0; r < rows; r += RS) {
+        const uint4 x = *reinterpret_cast<const uint4*>(src + r * D);
+        uint8_t* rowp = dst + r * 128;
+        *reinterpret_cast<uint4*>(rowp + dst_lo) =
+            make_uint4(pair(x.x, 0x1404), pair(x.x, 0x3424), pair(x.y, 0x1404), pair(x.y, 0x3424));
+        *reinterpret_cast<uint4*>(rowp + dst_hi) =
+            make_uint4(pair(x.z, 0x1404), pair(x.z, 0x3424), pair(x.w, 0x1404), pair(x.w, 0x3424));
       }
       fence_proxy_async_smem();  // the tensor cores read these bytes next
       __syncwarp();
