@@ -156,3 +156,14 @@ def test_pack_unpack_roundtrip(nK):
     t1, c1 = oracle.oracle_tables_bits(bits, 1, nK)
     t2, c2 = oracle.oracle_tables(m, 1)
     assert np.array_equal(t1, t2) and np.array_equal(c1, c2)
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama16k", "ctx128k"])
+def test_aligned_configs_last_live_block_is_the_diagonal(name):
+    """For block-aligned prefix and chunk the general rule gives the diagonal
+    block nPblk + qb, so the aligned configs' masks are what they always were."""
+    w = workloads.get_config(name)
+    last = workloads.last_live_block(w.prefix_len, w.chunk_len, w.block)
+    assert last.tolist() == (w.nPblk + np.arange(w.nQblk)).tolist()
+    live = workloads.causal_live(w.nPblk, w.nQblk, w.nKblk)
+    assert np.array_equal(live, workloads.causal_live(w.nPblk, w.nQblk, w.nKblk, last))
