@@ -284,9 +284,12 @@ __global__ void __launch_bounds__(128 + NT * 128, 1)
       const int u = blockIdx.x / p.n_splits;
       const UnitCoord uc = unit_coord(p, u);
       const int cnt = fused_group_table(p, uc, fent, nthreads);
-      if (p.tables_out && uc.qs == 0 && uc.hh == 0 && blockIdx.x % p.n_splits == 0) {
-        int32_t* trow_out = p.tables_out + (size_t)uc.g * uc.d.nKblk;
-        for (int e = threadIdx.x; e < uc.d.nKblk; e += nthreads) trow_out[e] = e < cnt ? fent[e] : -1;
+      if (uc.qs == 0 && uc.hh == 0 && blockIdx.x % p.n_splits == 0) {  // one CTA per group
+        if (p.tables_out) {
+          int32_t* trow_out = p.tables_out + (size_t)uc.g * uc.d.nKblk;
+          for (int e = threadIdx.x; e < uc.d.nKblk; e += nthreads)
+            trow_out[e] = e < cnt ? fent[e] : -1;
+        }
         if (threadIdx.x == 0 && p.counts_out) p.counts_out[uc.g] = cnt;
       }
       if (threadIdx.x == 0) {

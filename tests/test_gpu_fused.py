@@ -94,3 +94,16 @@ def test_fused_against_oracle(bsc, Hq, Hkv, d, B, P, L, dtype, S):
                                                x["V_pages"].double().numpy(),
                                                x["page_table"].numpy(), to, co, P)
         compare(O.float().cpu().numpy(), Lse.cpu().numpy(), Oo, Lo)
+
+
+def test_counts_out_without_tables_out(bsc):
+    w = workloads.Workload("c", 8, 2, 128, "bf16", 1024, 256, 64, "vslash", rho=0.1, corr=0.5,
+                           window=4, seed=5)
+    x = workloads.make_qkv_pages(w)
+    m = workloads.mask_for(w)
+    d = {k: v.cuda() for k, v in x.items()}
+    c = torch.full((w.Hkv,), 7, dtype=torch.int32, device="cuda")
+    bsc.chunk_attention_masked(d["Q"], d["K_pages"], d["V_pages"], d["page_table"], bits_of(m),
+                               w.prefix_len, counts_out=c)
+    _, co = oracle.oracle_tables(m, w.Hkv)
+    assert np.array_equal(c.cpu().numpy(), co)
