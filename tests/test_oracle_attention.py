@@ -30,23 +30,31 @@ def _val(s):
     return float(Fraction(s))
 
 
-def test_hand_derived_case():
-    g = json.load(open(os.path.join(GOLD, "attention_hand.json")))
+@pytest.mark.parametrize("fixture", ["attention_hand.json", "attention_unaligned_hand.json"])
+def test_hand_derived_case(fixture):
+    """Hand-derived values; the unaligned fixture has prefix 3 + chunk 2 at
+    block 2, so its last block holds one key and an empty slot."""
+    g = json.load(open(os.path.join(GOLD, fixture)))
     a = np.array([_val(x) for x in g["a"]])
     b = np.array([_val(x) for x in g["b"]])
     T = len(a)
-    K = math.sqrt(2.0) * np.stack([a, b], axis=1)           # logical keys [T, 2]
-    V = np.stack([np.arange(T, dtype=float), np.ones(T)], axis=1)
+    assert T == g["prefix_len"] + g["chunk_len"]
     pt = np.array(g["page_table"])
     B = g["block"]
-    Kp = np.zeros((len(pt), 1, B, 2))
-    Vp = np.zeros((len(pt), 1, B, 2))
+    nK = len(pt)
+    assert nK == -(-T // B)
+    K = np.zeros((nK * B, 2))                                # logical keys, empty slots 0
+    V = np.zeros((nK * B, 2))
+    K[:T] = math.sqrt(2.0) * np.stack([a, b], axis=1)
+    V[:T] = np.stack([np.arange(T, dtype=float), np.ones(T)], axis=1)
+    Kp = np.zeros((nK, 1, B, 2))
+    Vp = np.zeros((nK, 1, B, 2))
     for kb, page in enumerate(pt):
         Kp[page, 0] = K[kb * B:(kb + 1) * B]
         Vp[page, 0] = V[kb * B:(kb + 1) * B]
     Q = np.array(g["Q"])
     for case in g["cases"]:
-        tab = np.full((1, 2), -1)
+        tab = np.full((1, nK), -1)
         tab[0, :case["count"]] = case["table"]
         O, L = oracle.oracle_chunk_attention(Q, Kp, Vp, pt, tab, [case["count"]], g["prefix_len"])
         expL = np.array([_val(x) for x in case["LSE"]])
