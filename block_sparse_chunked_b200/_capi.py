@@ -123,11 +123,21 @@ def _out(name, t, like_device, dtype, numel):
     return t
 
 
-def _errp(err_flag):
-    """Pointer to the caller's device error word (int32 CUDA tensor), or None."""
+def _same_device(dev, **tensors):
+    """Every given tensor (None skipped) must live on `dev`: the kernels run on
+    that device and take raw pointers."""
+    for name, t in tensors.items():
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the call runs on {dev}")
+
+
+def _errp(err_flag, dev=None):
+    """Pointer to the caller's device error word (int32 CUDA tensor on `dev`), or None."""
     if err_flag is None:
         return None
     _need_cuda("err_flag", err_flag, (torch.int32,))
+    if dev is not None:
+        _same_device(dev, err_flag=err_flag)
     if err_flag.numel() < 1:
         raise ValueError("err_flag must hold one int32")
     return _ptr(err_flag)
@@ -154,8 +164,9 @@ def build_tables_batched(masks, Hkv, tables=None, counts=None):
         counts = torch.empty(nb, Hkv, dtype=torch.int32, device=masks.device)
     _out("tables", tables, masks.device, torch.int32, nb * Hkv * nK)
     _out("counts", counts, masks.device, torch.int32, nb * Hkv)
-    _ok(lib.ca_build_tables_batched(_ptr(masks), nb, Hq, Hkv, nQ, nK, _ptr(tables), _ptr(counts),
-                                    _stream()))
+    with torch.cuda.device(masks.device):
+        _ok(lib.ca_build_tables_batched(_ptr(masks), nb, Hq, Hkv, nQ, nK, _ptr(tables),
+                                        _ptr(counts), _stream()))
     return tables, counts
 
 
@@ -169,7 +180,9 @@ def build_tables(mask, Hkv, tables=None, counts=None):
         counts = torch.empty(Hkv, dtype=torch.int32, device=mask.device)
     _out("tables", tables, mask.device, torch.int32, Hkv * nK)
     _out("counts", counts, mask.device, torch.int32, Hkv)
-    _ok(lib.ca_build_tables(_ptr(mask), Hq, Hkv, nQ, nK, _ptr(tables), _ptr(counts), _stream()))
+    with torch.cuda.device(mask.device):
+        _ok(lib.ca_build_tables(_ptr(mask), Hq, Hkv, nQ, nK, _ptr(tables), _ptr(counts),
+                                _stream()))
     return tables, counts
 
 
@@ -186,8 +199,9 @@ def build_tables_bits(mask_bits, Hkv, nKblk, tables=None, counts=None):
         counts = torch.empty(nb, Hkv, dtype=torch.int32, device=mask_bits.device)
     _out("tables", tables, mask_bits.device, torch.int32, nb * Hkv * nKblk)
     _out("counts", counts, mask_bits.device, torch.int32, nb * Hkv)
-    _ok(lib.ca_build_tables_bits(_ptr(mask_bits), nb, Hq, Hkv, nQ, nKblk, _ptr(tables),
-                                 _ptr(counts), _stream()))
+    with torch.cuda.device(mask_bits.device):
+        _ok(lib.ca_build_tables_bits(_ptr(mask_bits), nb, Hq, Hkv, nQ, nKblk, _ptr(tables),
+                                     _ptr(counts), _stream()))
     return tables, counts
 
 
@@ -217,6 +231,8 @@ def chunk_attention(Q, K_pages, V_pages, page_table, tables, counts, prefix_len,
     _need_cuda("page_table", page_table, (torch.int32,), 1)
     _need_cuda("tables", tables, (torch.int32,), 2)
     _need_cuda("counts", counts, (torch.int32,), 1)
+    _same_device(Q.device, K_pages=K_pages, V_pages=V_pages, page_table=page_table,
+                 tables=tables, counts=counts)
     if K_pages.shape != V_pages.shape:
         raise ValueError("K_pages and V_pages must have the same shape")
     L, Hq, d = Q.shape
@@ -236,10 +252,12 @@ def chunk_attention(Q, K_pages, V_pages, page_table, tables, counts, prefix_len,
     _out("lse", lse, Q.device, torch.float32, Hq * L)
     ws_n = workspace_size(code, Hq, Hkv, d, B, L, prefix_len, num_pages, n_splits)
     workspace = _workspace(workspace, ws_n, Q.device)
-    _ok(lib.ca_chunk_attention(
-        _ptr(Q), _ptr(K_pages), _ptr(V_pages), code, num_pages, _ptr(page_table), _ptr(tables),
-        _ptr(counts), Hq, Hkv, d, B, L, prefix_len, _ptr(out), _ptr(lse),
-        _ptr(workspace) if ws_n else None, ws_n, n_splits, _errp(err_flag), _stream()))
+    with torch.cuda.device(Q.device):
+        _ok(lib.ca_chunk_attention(
+            _ptr(Q), _ptr(K_pages), _ptr(V_pages), code, num_pages, _ptr(page_table),
+            _ptr(tables), _ptr(counts), Hq, Hkv, d, B, L, prefix_len, _ptr(out), _ptr(lse),
+            _ptr(workspace) if ws_n else None, ws_n, n_splits, _errp(err_flag, Q.device),
+            _stream()))
     return out, lse
 
 
@@ -256,6 +274,8 @@ def chunk_attention_fp8(Q, K8, V8, K_scale, V_scale, page_table, tables, counts,
     _need_cuda("page_table", page_table, (torch.int32,), 1)
     _need_cuda("tables", tables, (torch.int32,), 2)
     _need_cuda("counts", counts, (torch.int32,), 1)
+    _same_device(Q.device, K8=K8, V8=V8, K_scale=K_scale, V_scale=V_scale,
+                 page_table=page_table, tables=tables, counts=counts)
     L, Hq, d = Q.shape
     num_pages, Hkv, B, d2 = K8.shape
     nK = -(-(prefix_len + L) // B)
@@ -273,10 +293,12 @@ def chunk_attention_fp8(Q, K8, V8, K_scale, V_scale, page_table, tables, counts,
     if ws_n == ctypes.c_size_t(-1).value:
         raise CompactAttnError(CA_ERR_ARG, "invalid shapes for ca_workspace_size_fp8")
     workspace = _workspace(workspace, ws_n, Q.device)
-    _ok(lib.ca_chunk_attention_fp8(
-        _ptr(Q), _ptr(K8), _ptr(V8), _ptr(K_scale), _ptr(V_scale), num_pages, _ptr(page_table),
-        _ptr(tables), _ptr(counts), Hq, Hkv, d, B, L, prefix_len, _ptr(out), _ptr(lse),
-        _ptr(workspace), ws_n, n_splits, _errp(err_flag), _stream()))
+    with torch.cuda.device(Q.device):
+        _ok(lib.ca_chunk_attention_fp8(
+            _ptr(Q), _ptr(K8), _ptr(V8), _ptr(K_scale), _ptr(V_scale), num_pages,
+            _ptr(page_table), _ptr(tables), _ptr(counts), Hq, Hkv, d, B, L, prefix_len,
+            _ptr(out), _ptr(lse), _ptr(workspace), ws_n, n_splits, _errp(err_flag, Q.device),
+            _stream()))
     return out, lse
 
 
@@ -291,6 +313,8 @@ def chunk_attention_masked(Q, K_pages, V_pages, page_table, mask_bits, prefix_le
     _need_cuda("V_pages", V_pages, (Q.dtype,), 4)
     _need_cuda("page_table", page_table, (torch.int32,), 1)
     _need_cuda("mask_bits", mask_bits, (torch.int32, torch.uint32), 3)
+    _same_device(Q.device, K_pages=K_pages, V_pages=V_pages, page_table=page_table,
+                 mask_bits=mask_bits, tables_out=tables_out, counts_out=counts_out)
     if K_pages.shape != V_pages.shape:
         raise ValueError("K_pages and V_pages must have the same shape")
     L, Hq, d = Q.shape
@@ -315,10 +339,12 @@ def chunk_attention_masked(Q, K_pages, V_pages, page_table, mask_bits, prefix_le
     if ws_n == ctypes.c_size_t(-1).value:
         raise CompactAttnError(CA_ERR_ARG, "invalid shapes for ca_workspace_size_masked")
     workspace = _workspace(workspace, ws_n, Q.device)
-    _ok(lib.ca_chunk_attention_masked(
-        _ptr(Q), _ptr(K_pages), _ptr(V_pages), code, num_pages, _ptr(page_table), _ptr(mask_bits),
-        Hq, Hkv, d, B, L, prefix_len, _ptr(tables_out), _ptr(counts_out), _ptr(out), _ptr(lse),
-        _ptr(workspace) if ws_n else None, ws_n, n_splits, _errp(err_flag), _stream()))
+    with torch.cuda.device(Q.device):
+        _ok(lib.ca_chunk_attention_masked(
+            _ptr(Q), _ptr(K_pages), _ptr(V_pages), code, num_pages, _ptr(page_table),
+            _ptr(mask_bits), Hq, Hkv, d, B, L, prefix_len, _ptr(tables_out), _ptr(counts_out),
+            _ptr(out), _ptr(lse), _ptr(workspace) if ws_n else None, ws_n, n_splits,
+            _errp(err_flag, Q.device), _stream()))
     return out, lse
 
 
@@ -339,6 +365,8 @@ def chunk_attention_varlen(Q, K_pages, V_pages, cu_q, prefix_len, page_table, cu
     for name, t in (("cu_q", cu_q), ("prefix_len", prefix_len), ("page_table", page_table),
                     ("cu_pages", cu_pages), ("tables", tables), ("counts", counts)):
         _need_cuda(name, t, (torch.int32,))
+    _same_device(Q.device, K_pages=K_pages, V_pages=V_pages, cu_q=cu_q, prefix_len=prefix_len,
+                 page_table=page_table, cu_pages=cu_pages, tables=tables, counts=counts)
     if K_pages.shape != V_pages.shape:
         raise ValueError("K_pages and V_pages must have the same shape")
     total_q, Hq, d = Q.shape
@@ -358,11 +386,12 @@ def chunk_attention_varlen(Q, K_pages, V_pages, cu_q, prefix_len, page_table, cu
     if ws_n == ctypes.c_size_t(-1).value:
         raise CompactAttnError(CA_ERR_ARG, "invalid shapes for ca_workspace_size_varlen")
     workspace = _workspace(workspace, ws_n, Q.device)
-    _ok(lib.ca_chunk_attention_varlen(
-        _ptr(Q), _ptr(K_pages), _ptr(V_pages), code, num_pages, S, total_q, _ptr(cu_q),
-        _ptr(prefix_len), max_kv_len, _ptr(page_table), _ptr(cu_pages), _ptr(tables),
-        _ptr(counts), Hq, Hkv, d, B, _ptr(out), _ptr(lse), _ptr(workspace), ws_n, n_splits,
-        _errp(err_flag), _stream()))
+    with torch.cuda.device(Q.device):
+        _ok(lib.ca_chunk_attention_varlen(
+            _ptr(Q), _ptr(K_pages), _ptr(V_pages), code, num_pages, S, total_q, _ptr(cu_q),
+            _ptr(prefix_len), max_kv_len, _ptr(page_table), _ptr(cu_pages), _ptr(tables),
+            _ptr(counts), Hq, Hkv, d, B, _ptr(out), _ptr(lse), _ptr(workspace), ws_n, n_splits,
+            _errp(err_flag, Q.device), _stream()))
     return out, lse
 
 
@@ -377,15 +406,26 @@ def append_kv(K_new, V_new, K_pages, V_pages, page_table, prefix_len, err_flag=N
     num_pages, Hkv2, B, d2 = K_pages.shape
     if V_new.shape != K_new.shape or V_pages.shape != K_pages.shape or Hkv2 != Hkv or d2 != d:
         raise ValueError("append_kv: inconsistent shapes")
-    _ok(lib.ca_append_kv(_ptr(K_new), _ptr(V_new), _DT[K_new.dtype], _ptr(K_pages), _ptr(V_pages),
-                         num_pages, _ptr(page_table), Hkv, d, B, prefix_len, L, _errp(err_flag),
-                         _stream()))
+    dev = K_new.device
+    _same_device(dev, V_new=V_new, K_pages=K_pages, V_pages=V_pages, page_table=page_table)
+    with torch.cuda.device(dev):
+        _ok(lib.ca_append_kv(_ptr(K_new), _ptr(V_new), _DT[K_new.dtype], _ptr(K_pages),
+                             _ptr(V_pages), num_pages, _ptr(page_table), Hkv, d, B, prefix_len, L,
+                             _errp(err_flag, dev), _stream()))
 
 
 def check(err_flag):
     """Synchronise, read and clear the device error word; raise on a device error."""
-    _ok(lib.ca_check(_errp(err_flag), _stream()))
+    if err_flag is None:
+        raise ValueError("check: err_flag is required")
+    p = _errp(err_flag)
+    with torch.cuda.device(err_flag.device):
+        _ok(lib.ca_check(p, _stream()))
 
 
 def wait_probe(err_flag, limit_us):
-    _ok(lib.ca_wait_probe(_errp(err_flag), int(limit_us), _stream()))
+    if err_flag is None:
+        raise ValueError("wait_probe: err_flag is required")
+    p = _errp(err_flag)
+    with torch.cuda.device(err_flag.device):
+        _ok(lib.ca_wait_probe(p, int(limit_us), _stream()))

@@ -140,6 +140,23 @@ def test_varlen_rejects_bad_arguments(bsc, kw, code):
 def test_check_and_probe_reject_null(bsc):
     assert bsc.lib.ca_check(None, None) == bsc.CA_ERR_ARG
     assert bsc.lib.ca_wait_probe(None, 10, None) == bsc.CA_ERR_ARG
+    with pytest.raises(ValueError):
+        bsc.check(None)
+    with pytest.raises(ValueError):
+        bsc.wait_probe(None, 10)
+
+
+def test_binding_device_check(bsc):
+    """Every tensor of a call must sit on the device the call runs on (the
+    kernels take raw pointers); a tensor elsewhere is refused before any launch."""
+    import torch
+    from block_sparse_chunked_b200 import _capi
+    dev = torch.device("cuda", 0)
+    _capi._same_device(torch.device("cpu"), a=torch.zeros(1), b=None)
+    with pytest.raises(ValueError, match="K_pages is on cpu"):
+        _capi._same_device(dev, K_pages=torch.zeros(1))
+    with pytest.raises(ValueError, match="err_flag"):
+        _capi._errp(torch.zeros(1, dtype=torch.int32), dev)   # not a CUDA tensor
 
 
 def test_accounting_dense_128k(bsc):
