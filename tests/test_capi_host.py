@@ -42,6 +42,36 @@ def test_library_exports_every_declared_symbol(bsc):
     assert set(header_symbols()) <= set(bsc.EXPORTS)
 
 
+def header_prototypes():
+    """name -> (return type, [parameter C types]) for every declaration."""
+    src = open(os.path.join(ROOT, "include", "compactattn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"^\s*(int|size_t)\s+(ca_\w+)\s*\(([^)]*)\)\s*;", src, flags=re.M):
+        params = [x.strip() for x in m.group(3).split(",") if x.strip() and x.strip() != "void"]
+        out[m.group(2)] = (m.group(1), params)
+    return out
+
+
+def test_binding_signatures_match_header(bsc):
+    """Each ctypes declaration has the header's arity and, parameter by
+    parameter, a matching kind: pointer -> c_void_p / c_char_p, int -> c_int,
+    size_t -> c_size_t.  (A drift here would pass wrong values to the GPU.)"""
+    protos = header_prototypes()
+    assert set(protos) == set(header_symbols())
+    for name, (ret, params) in protos.items():
+        res, args = bsc.EXPORTS[name]
+        assert res is (ctypes.c_int if ret == "int" else ctypes.c_size_t), name
+        assert len(args) == len(params), (name, len(args), len(params))
+        for a, ctype in zip(args, params):
+            if "*" in ctype:
+                assert a in (ctypes.c_void_p, ctypes.c_char_p), (name, ctype)
+            elif re.match(r"(const\s+)?size_t\b", ctype):
+                assert a is ctypes.c_size_t, (name, ctype)
+            else:
+                assert re.match(r"(const\s+)?int\b", ctype) and a is ctypes.c_int, (name, ctype)
+
+
 def test_version(bsc):
     assert bsc.version() == 100
 
