@@ -297,7 +297,6 @@ def cpu_oracle_sample(w, x, mask, budget_s=12.0, stride=None):
     """Time the float64 oracle (tables in full + attention on a row sample) on host cores."""
     import numpy as np
 
-    import block_sparse_chunked_b200 as bsc
     import oracle
     t0 = time.perf_counter()
     t, c = oracle.oracle_tables(mask, w.Hkv)
@@ -316,7 +315,10 @@ def cpu_oracle_sample(w, x, mask, budget_s=12.0, stride=None):
                        w.prefix_len, rows)
     dt = time.perf_counter() - t0
     flops = sum(4.0 * w.head_dim * w.block * live[h // G][i // w.block] for h, i in rows)
-    tot_flops = bsc.selected_flops(t, c, w.Hq, w.nPblk, w.nQblk, w.block, w.head_dim)
+    # total selected FLOPs of the chunk, from the oracle's own tables (this leg
+    # must not load the CUDA library)
+    tot_flops = sum(4.0 * w.head_dim * w.block * w.block * int(live[h // G].sum())
+                    for h in range(w.Hq))
     try:
         from threadpoolctl import threadpool_info
         blas = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])

@@ -195,7 +195,7 @@ cudaError_t launch_build_tables(const uint8_t* mask, int nb, int Hq, int Hkv, in
   // Cluster size: enough CTAs for ~CA_BUILD_CTAS_PER_SM per SM over all (mask, group) units,
   // at most 8 per cluster and at least 256 columns per CTA.
   const long long units = (long long)nb * Hkv;
-  int C = (int)((CA_BUILD_CTAS_PER_SM * 148 + units - 1) / units);
+  int C = (int)((CA_BUILD_CTAS_PER_SM * num_sms() + units - 1) / units);
   C = C > 8 ? 8 : C;
   const int cmax = (nKblk + 255) / 256;
   C = C > cmax ? cmax : C;

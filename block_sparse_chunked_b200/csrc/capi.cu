@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -54,7 +55,6 @@ EncodeTiledFn encoder() {
   return fn;
 }
 
-constexpr int kSMs = 148;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per pipeline wait
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -89,13 +89,14 @@ bool plan_mode(Plan& pl, long long units, int max_stages, int n_splits, bool all
   // all units' KV stages (at least ~4 stages per CTA).  (At 256 units on 148
   // SMs the persistent grid measured 5% slower than one CTA per unit: the
   // piece boundaries and the merge cost more than the balance gains.)
-  pl.persistent = (allow_persistent && n_splits <= 0 && units < kSMs && units <= kMaxPersistentUnits)
+  const int sms = num_sms();
+  pl.persistent = (allow_persistent && n_splits <= 0 && units < sms && units <= kMaxPersistentUnits)
                       ? 1 : 0;
   if (n_splits <= 0 && !pl.persistent) n_splits = 1;
   pl.sk_ctas = 0;
   if (pl.persistent) {
     const long long stages = units * max_stages;
-    pl.sk_ctas = (int)std::max<long long>(1, std::min<long long>(kSMs, stages / 4));
+    pl.sk_ctas = (int)std::max<long long>(1, std::min<long long>(sms, stages / 4));
     pl.n_splits = 1;
     return true;
   }
@@ -190,6 +191,32 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 }  // namespace
 
 void set_last_error(const char* msg) { g_last_error = msg ? msg : ""; }
+
+// Streaming multiprocessors of the calling thread's current device: the
+// persistent grid and the automatic split plan are sized from it.  Without a
+// usable device (a host-only size query) the B200's 148 is assumed; a plan made
+// that way is checked again by the launching call, which needs the workspace
+// its own device's plan asks for.
+int num_sms() {
+  static std::atomic<int> cache[64];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    (void)cudaGetLastError();
+    return 148;
+  }
+  if (dev < 64) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    return 148;
+  }
+  if (dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
 
 }  // namespace ca
 
@@ -427,7 +454,8 @@ bool plan_masked(int Hq, int Hkv, int head_dim, int block, int chunk_len, int pr
   if (d.nKblk > max_nKblk) return false;
   const int max_stages = (d.nKblk + pl.spb - 1) / pl.spb;
   int S = n_splits;
-  if (S <= 0) S = pl.units >= kSMs ? 1 : (2 * kSMs + pl.units - 1) / pl.units;
+  const int sms = num_sms();
+  if (S <= 0) S = pl.units >= sms ? 1 : (2 * sms + pl.units - 1) / pl.units;
   if (S > 16 && n_splits <= 0) S = 16;
   return plan_mode(pl, pl.units, max_stages, S, false);
 }

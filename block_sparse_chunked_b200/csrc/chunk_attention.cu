@@ -1223,7 +1223,7 @@ cudaError_t launch_split_combine(const float* Opart, const float* LSEpart, int n
 cudaError_t launch_cast_f32_bf16(const float* src, void* dst, size_t n, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   size_t blocks = (n / 4 + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks > (size_t)num_sms() * 16) blocks = (size_t)num_sms() * 16;
   if (blocks < 1) blocks = 1;
   cast_f32_bf16_kernel<<<(unsigned)blocks, 256, 0, st>>>(src, reinterpret_cast<__nv_bfloat16*>(dst), n);
   return cudaGetLastError();
@@ -1233,7 +1233,7 @@ cudaError_t launch_split_f32_bf16(const float* src, void* hi, void* lo, size_t n
                                   cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   size_t blocks = (n + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks > (size_t)num_sms() * 16) blocks = (size_t)num_sms() * 16;
   split_f32_bf16_kernel<<<(unsigned)blocks, 256, 0, st>>>(
       src, reinterpret_cast<__nv_bfloat16*>(hi), reinterpret_cast<__nv_bfloat16*>(lo), n);
   return cudaGetLastError();
@@ -1251,7 +1251,7 @@ cudaError_t launch_varlen_setup(const int32_t* cu_q, const int32_t* prefix_len,
 cudaError_t launch_cast_bf16_f16(const void* src, void* dst, size_t n, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   size_t blocks = (n + 255) / 256;
-  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks > (size_t)num_sms() * 16) blocks = (size_t)num_sms() * 16;
   cast_bf16_f16_kernel<<<(unsigned)blocks, 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(src), static_cast<__half*>(dst), n);
   return cudaGetLastError();

@@ -84,6 +84,10 @@ cudaError_t launch_split_f32_bf16(const float* src, void* hi, void* lo, size_t n
                                   cudaStream_t st);
 cudaError_t launch_wait_probe(int32_t* err, unsigned long long limit_ns, cudaStream_t st);
 
+// Streaming multiprocessors of the calling thread's current device (148 when
+// no device can be queried).
+int num_sms();
+
 // Record a message for ca_last_error() on the calling thread.
 void set_last_error(const char* msg);
 

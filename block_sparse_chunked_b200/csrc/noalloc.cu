@@ -17,6 +17,7 @@
 // was written by the same call).  Calls whose kernels overlap on the GPU —
 // on two streams, or from two host threads — race on the array and give
 // wrong results: serialise them.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -33,11 +34,51 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device, looked up once
-// per device.  In host code the array's name only stands in for the symbol;
-// the kernel needs the address cudaGetSymbolAddress returns for this device.
+// Per device: the unique id of the context the address was looked up in, and
+// the address.  A reset of the device (cudaDeviceReset) destroys the context
+// and the next one reloads the module, so the array may then sit at another
+// address; a cached address is only reused while the device's current context
+// is the one it came from.  Context ids (cuCtxGetId) are never reused within a
+// process, unlike context handles.
+struct ScratchAddr {
+  unsigned long long ctx_id = 0;
+  bool valid = false;
+  void* ptr = nullptr;
+};
+ScratchAddr g_scratch[kMaxDevices];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+void* driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    return p;
+  return nullptr;
+}
+
+// Unique id of the calling thread's current context; false if there is none.
+bool current_ctx_id(unsigned long long* id) {
+  static std::once_flag once;
+  static CtxGetCurrentFn get = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  std::call_once(once, [] {
+    get = reinterpret_cast<CtxGetCurrentFn>(driver_fn("cuCtxGetCurrent"));
+    get_id = reinterpret_cast<CtxGetIdFn>(driver_fn("cuCtxGetId"));
+  });
+  CUcontext ctx = nullptr;
+  if (!get || !get_id || get(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch array in the current device's current
+// context.  In host code the array's name only stands in for the symbol; the
+// kernels need the address cudaGetSymbolAddress returns for this device.  The
+// lookup runs on the first call per device and again on the first call after
+// that device's context has changed (a reset).
 int scratch_address(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -45,17 +86,28 @@ int scratch_address(void** out) {
     ca::set_last_error("ca_chunk_attention_noalloc: no usable current device");
     return CA_ERR_LAUNCH;
   }
+  unsigned long long id = 0;
+  const bool have_id = current_ctx_id(&id);
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
+  ScratchAddr& c = g_scratch[dev];
+  if (!have_id || !c.valid || c.ctx_id != id) {
+    // (the lookup also binds the device's primary context to this thread when
+    // no context is current yet; the context is read again after it)
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p) {
       ca::set_last_error("ca_chunk_attention_noalloc: cudaGetSymbolAddress of the scratch failed");
       return CA_ERR_LAUNCH;
     }
-    g_scratch_addr[dev] = p;
+    if (!current_ctx_id(&id)) {
+      ca::set_last_error("ca_chunk_attention_noalloc: cannot identify the current CUDA context");
+      return CA_ERR_LAUNCH;
+    }
+    c.ctx_id = id;
+    c.valid = true;
+    c.ptr = p;
   }
-  *out = g_scratch_addr[dev];
+  *out = c.ptr;
   return CA_OK;
 }
 

@@ -283,8 +283,11 @@ int ca_chunk_attention_fp8(const void* Q, const uint8_t* K_pages, const uint8_t*
  *     CA_ERR_WORKSPACE (nothing is launched); n_splits <= 0 picks the split
  *     as ca_chunk_attention does.
  *   - The first call on each device looks up the scratch array's device
- *     address (cudaGetSymbolAddress, with that device current); make that
- *     first call before any stream capture.
+ *     address (cudaGetSymbolAddress, with that device current) and keeps it
+ *     for that device's context; make that first call before any stream
+ *     capture.  The address is valid for one context lifetime only: after
+ *     cudaDeviceReset (or any new context on the device) the next call looks
+ *     it up again, so that call, too, belongs before any capture.
  *   - All calls on a device share the scratch and it keeps the last call's
  *     contents (nothing in it needs to start at zero).  Calls whose kernels
  *     overlap on the GPU race on it: do not run two at once on one device.

@@ -254,19 +254,3 @@ def test_sweep_chunks_sampled_rows(bsc, c):
                                 x["page_table"].numpy(), t, cn, w.prefix_len, rows)
     compare(np.stack([O[i, h] for h, i in rows]), np.array([Lg[h, i] for h, i in rows]), Oo, Lo)
     assert np.all(np.isfinite(Lg))
-
-
-@pytest.mark.parametrize("rho,corr,block", [(1.0, 0.0, 64), (0.05, 0.0, 128), (0.2, 1.0, 64),
-                                            (0.1, 0.5, 128)])
-def test_density_cells_sampled_rows(bsc, rho, corr, block):
-    """64K context, 2048-token chunk: density / within-group correlation cells, B 64 and 128."""
-    w = workloads.density_cell(rho, corr, block=block)
-    x = workloads.make_qkv_pages(w)
-    m = workloads.mask_for(w)
-    O, Lg, t, c = gpu_run(bsc, w, x, m)
-    if rho >= 1.0:
-        assert c.tolist() == [w.nKblk] * w.Hkv
-    rows = sample_rows(w, seed=3, ntok=6)[::2]
-    Oo, Lo = oracle.oracle_rows(x["Q"].double().numpy(), x["K_pages"], x["V_pages"],
-                                x["page_table"].numpy(), t, c, w.prefix_len, rows)
-    compare(np.stack([O[i, h] for h, i in rows]), np.array([Lg[h, i] for h, i in rows]), Oo, Lo)

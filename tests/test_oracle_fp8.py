@@ -70,3 +70,64 @@ def test_fp8_oracle_is_the_oracle_on_decoded_pages():
                                                x["page_table"].numpy(), t, c, w.prefix_len)
     np.testing.assert_allclose(O3, 2 * O, rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(L3, L, rtol=0, atol=1e-12)
+
+
+def _fp8_case():
+    """A small E4M3 cache with scales spread over (page, head) so that a wrong
+    tile or a dropped scale moves the result: 3 KV heads, 11 pages."""
+    w = workloads.Workload("qr", 6, 3, 16, "fp32", 144, 32, 16, "bernoulli", rho=0.35, seed=5)
+    x = workloads.make_qkv_pages(w)
+    m = workloads.mask_for(w)
+    t, c = oracle.oracle_tables(m, w.Hkv)
+    K8, sK = workloads.quantize_pages_e4m3(x["K_pages"])
+    V8, sV = workloads.quantize_pages_e4m3(x["V_pages"])
+    rng = np.random.default_rng(7)
+    sK = sK.numpy() * rng.uniform(0.5, 4.0, sK.shape)
+    sV = sV.numpy() * rng.uniform(0.5, 4.0, sV.shape)
+    rows = [(h, i) for h in range(w.Hq) for i in range(w.chunk_len)]
+    return w, x, t, c, K8.numpy(), V8.numpy(), sK, sV, rows
+
+
+def test_rows_fp8_matches_full_fp8_oracle_row_by_row():
+    """oracle_rows_fp8 (pages decoded one (page, head) tile at a time, the
+    checker of the full-size E4M3 GPU test) equals oracle_chunk_attention_fp8 on
+    every (head, token) row of a small cache."""
+    w, x, t, c, K8, V8, sK, sV, rows = _fp8_case()
+    Q = x["Q"].double().numpy()
+    pt = x["page_table"].numpy()
+    O, L = oracle.oracle_chunk_attention_fp8(Q, K8, V8, sK, sV, pt, t, c, w.prefix_len)
+    Or, Lr = oracle.oracle_rows_fp8(Q, K8, V8, sK, sV, pt, t, c, w.prefix_len, rows)
+    np.testing.assert_allclose(Or, np.stack([O[i, h] for h, i in rows]), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(Lr, np.array([L[h, i] for h, i in rows]), rtol=0, atol=1e-12)
+
+
+class _SwappedTile(oracle.fp8._DecodedPages):
+    def __getitem__(self, idx):  # planted mistake: (head, page) instead of (page, head)
+        p, g = idx
+        return oracle.decode_e4m3(self.codes[g % self.shape[0], p % self.shape[1]]) * \
+            self.scale[p, g]
+
+
+class _DroppedScale(oracle.fp8._DecodedPages):
+    def __getitem__(self, idx):  # planted mistake: the tile's scale left out
+        p, g = idx
+        return oracle.decode_e4m3(self.codes[p, g])
+
+
+class _WrongScale(oracle.fp8._DecodedPages):
+    def __getitem__(self, idx):  # planted mistake: another head's scale
+        p, g = idx
+        return oracle.decode_e4m3(self.codes[p, g]) * self.scale[p, (g + 1) % self.shape[1]]
+
+
+@pytest.mark.parametrize("planted", [_SwappedTile, _DroppedScale, _WrongScale])
+def test_rows_fp8_pin_catches_planted_mistakes(planted):
+    w, x, t, c, K8, V8, sK, sV, rows = _fp8_case()
+    Q = x["Q"].double().numpy()
+    pt = x["page_table"].numpy()
+    O, L = oracle.oracle_chunk_attention_fp8(Q, K8, V8, sK, sV, pt, t, c, w.prefix_len)
+    Ob, Lb = oracle.oracle_rows(Q, planted(K8, sK), planted(V8, sV), pt, t, c, w.prefix_len,
+                                rows)
+    Of = np.stack([O[i, h] for h, i in rows])
+    Lf = np.array([L[h, i] for h, i in rows])
+    assert np.abs(Ob - Of).max() > 1e-3 or np.abs(Lb - Lf).max() > 1e-3
