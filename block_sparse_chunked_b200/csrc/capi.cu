@@ -64,20 +64,76 @@ constexpr int kMaxPersistentUnits = 2048;  // units whose schedule a CTA keeps i
 struct Plan {
   int G, HPU, NT, nhalves, spb, n_splits;
   int units, persistent, sk_ctas;
+  int tile;                          // 1: the one-tile kernel (bf16 pages and Q)
+  int tail_start, tail_k, n_tail;    // tile kernel: the split last partial wave
 };
 
-// Heads -> tiles: a unit stacks up to four heads of a group over a 64-token
-// span (two heads per 128-row tile).
-bool plan_heads(int Hq, int Hkv, int head_dim, int block, Plan& pl) {
+// Heads -> tiles.  Two-tile kernel: a unit stacks up to four heads of a group
+// over a 64-token span (two heads per 128-row tile).  One-tile kernel: a unit
+// is two heads of a group over a 64-token span, one 128-row tile.
+bool plan_heads(int Hq, int Hkv, int head_dim, int block, Plan& pl, bool tile = false) {
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return false;
   if (head_dim != 64 && head_dim != 128) return false;
   if (block != 64 && block != 128) return false;
   pl.G = Hq / Hkv;
-  pl.HPU = pl.G < 4 ? pl.G : 4;
-  pl.NT = (pl.HPU + 1) / 2;
-  pl.nhalves = (pl.G + pl.HPU - 1) / pl.HPU;
+  pl.tile = tile ? 1 : 0;
+  if (tile) {
+    pl.HPU = pl.G < 2 ? pl.G : 2;
+    pl.NT = 1;
+    pl.nhalves = (pl.G + 1) / 2;
+  } else {
+    pl.HPU = pl.G < 4 ? pl.G : 4;
+    pl.NT = (pl.HPU + 1) / 2;
+    pl.nhalves = (pl.G + pl.HPU - 1) / pl.HPU;
+  }
   pl.spb = 128 / block;
+  pl.tail_start = 0;
+  pl.tail_k = 1;
+  pl.n_tail = 0;
   return true;
+}
+
+// Work mode of the one-tile kernel for `units` units of at most `max_stages`
+// KV stages each (one CTA per SM).  n_splits > 0: every unit in that many KV
+// pieces.  Automatic (n_splits <= 0): with fewer units than SMs, every unit in
+// floor(SMs / units) pieces (at most 16), so that one wave fills the SMs;
+// otherwise one CTA per unit, and when the units are known exactly the r
+// units of the last partial wave run as k pieces each, k the largest with
+// r * k <= SMs (at most 4): the last wave then takes 1/k of a unit's time.
+bool plan_mode_tile(Plan& pl, long long units, int max_stages, int n_splits, bool exact_units) {
+  if (units > 0x7fffffffLL) return false;
+  pl.units = (int)units;
+  pl.persistent = 0;
+  pl.sk_ctas = 0;
+  pl.tail_start = (int)units;
+  pl.tail_k = 1;
+  pl.n_tail = 0;
+  const long long sms = num_sms();
+  long long S = n_splits;
+  if (S <= 0) {
+    S = units > 0 && units < sms ? std::min<long long>(16, std::max<long long>(1, sms / units)) : 1;
+    const long long r = units % sms;
+    if (exact_units && units >= sms && r > 0) {
+      const int k = (int)std::min<long long>({4, sms / r, (long long)max_stages});
+      if (k >= 2) {
+        pl.tail_k = k;
+        pl.n_tail = (int)r;
+        pl.tail_start = (int)(units - r);
+      }
+    }
+  }
+  if (S > max_stages) S = max_stages;
+  if (S < 1) S = 1;
+  if (units * S > 0x7fffffffLL) return false;
+  pl.n_splits = (int)S;
+  return true;
+}
+
+// Grid of an attention launch for plan pl.
+int plan_grid(const Plan& pl) {
+  if (pl.persistent) return pl.sk_ctas;
+  if (pl.tile && pl.tail_k > 1) return pl.tail_start + pl.n_tail * pl.tail_k;
+  return pl.units * pl.n_splits;
 }
 
 // Work mode for `units` units of at most `max_stages` KV stages each.
@@ -112,8 +168,8 @@ bool plan_mode(Plan& pl, long long units, int max_stages, int n_splits, bool all
 // alignment needed: masks hold Q-blocks of the chunk's tokens and KV blocks
 // of the sequence's positions).
 bool plan(int Hq, int Hkv, int head_dim, int block, int chunk_len, int prefix_len, int n_splits,
-          Plan& pl, SeqDesc& d) {
-  if (!plan_heads(Hq, Hkv, head_dim, block, pl)) return false;
+          Plan& pl, SeqDesc& d, bool tile = false) {
+  if (!plan_heads(Hq, Hkv, head_dim, block, pl, tile)) return false;
   if (chunk_len < 1 || prefix_len < 0 || (long long)prefix_len + chunk_len > 0x7fffffffLL)
     return false;
   d.q_start = 0;
@@ -126,12 +182,13 @@ bool plan(int Hq, int Hkv, int head_dim, int block, int chunk_len, int prefix_le
   d.seq = 0;
   const long long units = (long long)Hkv * pl.nhalves * d.nqs;
   const int max_stages = (d.nKblk + pl.spb - 1) / pl.spb;
+  if (tile) return plan_mode_tile(pl, units, max_stages, n_splits, true);
   return plan_mode(pl, units, max_stages, n_splits, true);
 }
 
 struct WsLayout {
   size_t opart = 0, lsepart = 0, q = 0, qlo = 0, k = 0, v = 0, sched = 0, osk = 0, lsesk = 0,
-         seqs = 0, nunits = 0, q16 = 0, esc = 0, total = 0;
+         seqs = 0, nunits = 0, q16 = 0, esc = 0, otail = 0, lsetail = 0, total = 0;
 };
 
 // rows = rows of Q / O; num_seqs > 0 reserves the batched call's descriptors.
@@ -154,6 +211,13 @@ WsLayout ws_layout(int dtype, int Hq, int Hkv, int D, int B, long long rows, int
     off = align256(off + 2 * (size_t)pl.sk_ctas * trows * D * 4);
     w.lsesk = off;
     off = align256(off + 2 * (size_t)pl.sk_ctas * trows * 4);
+  }
+  if (pl.tile && pl.tail_k > 1) {
+    const size_t pieces = (size_t)pl.n_tail * pl.tail_k;
+    w.otail = off;
+    off = align256(off + pieces * 128 * D * 4);
+    w.lsetail = off;
+    off = align256(off + pieces * 128 * 4);
   }
   if (S > 1) {
     w.opart = off;
@@ -184,6 +248,18 @@ WsLayout ws_layout(int dtype, int Hq, int Hkv, int D, int B, long long rows, int
 // Units bound of a batched call: sum_s ceil(L_s / 64) <= total_q / 64 + num_seqs.
 long long varlen_units_bound(int total_q, int num_seqs, int Hkv, int nhalves) {
   return ((long long)(total_q + 63) / 64 + num_seqs) * Hkv * nhalves;
+}
+
+// Plan of a batched call (the exact unit count is only known on the device:
+// the plan is made for the bound, and surplus CTAs leave at once).
+bool plan_varlen(int Hq, int Hkv, int head_dim, int block, int dtype, int num_seqs, int total_q,
+                 int max_kv_len, int n_splits, Plan& pl) {
+  const bool tile = dtype == CA_DTYPE_BF16;
+  if (!plan_heads(Hq, Hkv, head_dim, block, pl, tile)) return false;
+  const int max_stages = std::max(1, (max_kv_len + 127) / 128);
+  const long long bound = varlen_units_bound(total_q, num_seqs, Hkv, pl.nhalves);
+  if (tile) return plan_mode_tile(pl, bound, max_stages, n_splits, false);
+  return plan_mode(pl, bound, max_stages, n_splits, false);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -279,7 +355,9 @@ size_t ca_workspace_size(int dtype, int Hq, int Hkv, int head_dim, int block, in
   Plan pl;
   SeqDesc d;
   if (dtype != CA_DTYPE_BF16 && dtype != CA_DTYPE_FP32) return (size_t)-1;
-  if (!plan(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl, d)) return (size_t)-1;
+  if (!plan(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl, d,
+            dtype == CA_DTYPE_BF16))
+    return (size_t)-1;
   if (num_pages < d.nKblk) return (size_t)-1;
   return ws_layout(dtype, Hq, Hkv, head_dim, block, chunk_len, num_pages, pl).total;
 }
@@ -289,10 +367,7 @@ size_t ca_workspace_size_varlen(int dtype, int Hq, int Hkv, int head_dim, int bl
   Plan pl;
   if (dtype != CA_DTYPE_BF16 && dtype != CA_DTYPE_FP32) return (size_t)-1;
   if (num_seqs < 1 || total_q < 0 || max_kv_len < 0 || num_pages < 1) return (size_t)-1;
-  if (!plan_heads(Hq, Hkv, head_dim, block, pl)) return (size_t)-1;
-  const int max_stages = std::max(1, (max_kv_len + 127) / 128);
-  if (!plan_mode(pl, varlen_units_bound(total_q, num_seqs, Hkv, pl.nhalves), max_stages,
-                 n_splits, false))
+  if (!plan_varlen(Hq, Hkv, head_dim, block, dtype, num_seqs, total_q, max_kv_len, n_splits, pl))
     return (size_t)-1;
   return ws_layout(dtype, Hq, Hkv, head_dim, block, total_q, num_pages, pl, num_seqs).total;
 }
@@ -366,6 +441,11 @@ int run_attention(const char* who, const void* Q, const void* K_pages, const voi
                   which ? "V" : "K", (int)r);
   }
 
+  p.tail_start = pl.tail_start;
+  p.tail_k = pl.tail_k;
+  p.n_tail = pl.n_tail;
+  p.Otail = pl.tail_k > 1 ? reinterpret_cast<float*>(ws + wl.otail) : nullptr;
+  p.LSEtail = pl.tail_k > 1 ? reinterpret_cast<float*>(ws + wl.lsetail) : nullptr;
   p.Opart = pl.n_splits > 1 ? reinterpret_cast<float*>(ws + wl.opart) : nullptr;
   p.LSEpart = pl.n_splits > 1 ? reinterpret_cast<float*>(ws + wl.lsepart) : nullptr;
   p.persistent = pl.persistent;
@@ -386,8 +466,11 @@ int run_attention(const char* who, const void* Q, const void* K_pages, const voi
   p.out_f32 = dtype == CA_DTYPE_FP32 ? 1 : 0;  // E4M3 pages: O is bf16
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   p.wait_ns = kWaitNs;
-  e = launch_chunk_attention(tq, tqlo, tk, tv, p, D, pl.NT, dtype == CA_DTYPE_FP32, kv8, grid,
-                             st);
+  if (pl.tile)
+    e = launch_chunk_attention_tile(tq, tk, tv, p, D, grid, st);
+  else
+    e = launch_chunk_attention(tq, tqlo, tk, tv, p, D, pl.NT, dtype == CA_DTYPE_FP32, kv8, grid,
+                               st);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   if (pl.persistent) {
     e = launch_sk_combine(p, D, pl.NT, st);
@@ -415,7 +498,8 @@ int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, 
     return fail(CA_ERR_ARG, "ca_chunk_attention: block=%d must be 64 or 128", block);
   Plan pl;
   SeqDesc d;
-  if (!plan(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl, d))
+  if (!plan(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl, d,
+            dtype == CA_DTYPE_BF16))
     return fail(CA_ERR_ARG,
                 "ca_chunk_attention: unsupported shape Hq=%d Hkv=%d head_dim=%d block=%d "
                 "chunk_len=%d prefix_len=%d",
@@ -439,7 +523,12 @@ int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, 
   p.seqs = nullptr;
   p.seq0 = d;
   p.num_seqs = 1;
-  const int grid = pl.persistent ? pl.sk_ctas : pl.units * pl.n_splits;
+  // When the prefix dominates, every span of a group sees nearly the same
+  // blocks and costs the same: run the units group by group, so that the pages
+  // in flight at one time are those of a few groups and stay in L2 for all the
+  // spans that read them.  Otherwise later spans (more blocks) go first.
+  p.unit_order = (pl.tile && (long long)prefix_len >= 2LL * chunk_len) ? 1 : 0;
+  const int grid = plan_grid(pl);
   return run_attention("ca_chunk_attention", Q, K_pages, V_pages, dtype, num_pages, Hq, Hkv,
                        head_dim, block, chunk_len, pl, wl, static_cast<uint8_t*>(workspace), grid,
                        p, static_cast<cudaStream_t>(stream));
@@ -595,9 +684,7 @@ int ca_chunk_attention_varlen(const void* Q, const void* K_pages, const void* V_
   if (!plan_heads(Hq, Hkv, head_dim, block, pl))
     return fail(CA_ERR_ARG, "%s: unsupported shape Hq=%d Hkv=%d head_dim=%d block=%d", who, Hq,
                 Hkv, head_dim, block);
-  const int max_stages = std::max(1, (max_kv_len + 127) / 128);
-  if (!plan_mode(pl, varlen_units_bound(total_q, num_seqs, Hkv, pl.nhalves), max_stages,
-                 n_splits, false))
+  if (!plan_varlen(Hq, Hkv, head_dim, block, dtype, num_seqs, total_q, max_kv_len, n_splits, pl))
     return fail(CA_ERR_ARG, "%s: too many work units", who);
   if (!aligned16(Q) || !aligned16(K_pages) || !aligned16(V_pages) || !aligned16(O))
     return fail(CA_ERR_ARG, "%s: Q, K_pages, V_pages and O must be 16-byte aligned", who);
@@ -624,7 +711,7 @@ int ca_chunk_attention_varlen(const void* Q, const void* K_pages, const void* V_
   p.seqs = seqs;
   p.seq0 = SeqDesc{};
   p.num_seqs = num_seqs;
-  const int grid = pl.units * pl.n_splits;
+  const int grid = plan_grid(pl);
   return run_attention(who, Q, K_pages, V_pages, dtype, num_pages, Hq, Hkv, head_dim, block,
                        total_q, pl, wl, ws, grid, p, st);
 }

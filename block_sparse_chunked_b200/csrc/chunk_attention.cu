@@ -40,6 +40,7 @@
 #include <cstdint>
 
 #include "compactattn.h"
+#include "attn_common.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -48,10 +49,6 @@ namespace ca {
 constexpr int kStageKeys = 128;
 
 
-
-__device__ __forceinline__ void set_flag(int32_t* err, int f) {
-  if (err) atomicOr(err, f);
-}
 
 // QSPLIT: Q is given as two bf16 terms (hi + lo) of an fp32 input and
 // S = Q_hi K^T + Q_lo K^T, which removes the rounding error of Q (the error
@@ -87,78 +84,6 @@ struct Smem {
   static constexpr int kBytes = kSchedOff + (KV8 ? 0 : (2 * 2048 + 1 + 32) * 4);
   static constexpr int kAlloc = kBytes + 1024;          // slack for 1024-B alignment
 };
-
-// Warp-uniform bounded wait.  Returns false (and flags / aborts) on expiry.
-__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, const AttnParams& p,
-                                          volatile int* abort_flag) {
-  bool ok = (*abort_flag == 0) && mbar_wait(bar, parity, p.wait_ns);
-  ok = __all_sync(0xffffffffu, ok);
-  if (!ok) {
-    if ((threadIdx.x & 31) == 0 && *abort_flag == 0) {
-      *abort_flag = 1;
-      set_flag(p.err, CA_FLAG_TIMEOUT);
-    }
-  }
-  return ok;
-}
-
-// Number of work units whose stage counts a persistent CTA keeps in shared memory.
-constexpr int kMaxUnits = 2048;
-
-// The sequence that owns unit u.
-__device__ __forceinline__ SeqDesc seq_of(const AttnParams& p, int u) {
-  if (p.seqs == nullptr) return p.seq0;
-  int lo = 0, hi = p.num_seqs - 1;  // last sequence with unit_start <= u
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (p.seqs[mid].unit_start <= u) lo = mid;
-    else hi = mid - 1;
-  }
-  return p.seqs[lo];
-}
-
-// Unit u -> (sequence, group, 64-token query span, head slice); within a
-// sequence, later query spans (more causal blocks) first.
-struct UnitCoord {
-  SeqDesc d;
-  int g, qs, hh;
-};
-__device__ __forceinline__ UnitCoord unit_coord(const AttnParams& p, int u) {
-  UnitCoord c;
-  c.d = seq_of(p, u);
-  const int loc = u - c.d.unit_start;
-  const int per_qs = p.Hkv * p.nhalves;
-  c.qs = c.d.nqs - 1 - loc / per_qs;
-  c.g = (loc % per_qs) / p.nhalves;
-  c.hh = (loc % per_qs) % p.nhalves;
-  return c;
-}
-
-__device__ __forceinline__ const int32_t* table_row(const AttnParams& p, const UnitCoord& c) {
-  return p.tables + (size_t)c.d.pt_off * p.Hkv + (size_t)c.g * c.d.nKblk;
-}
-
-// Live table entries of unit u: the entries whose block can hold a key visible
-// to the span's last query (kb * B <= P + last token), a prefix of the
-// ascending row (binary search).
-__device__ __forceinline__ int unit_live(const AttnParams& p, int u) {
-  const UnitCoord c = unit_coord(p, u);
-  const int t_last = min(c.qs * 64 + 63, c.d.L - 1);
-  const int last_kb = (c.d.P + t_last) / p.B;
-  const int32_t* trow = table_row(p, c);
-  int cnt = p.counts[(size_t)c.d.seq * p.Hkv + c.g];
-  if (cnt < 0 || cnt > c.d.nKblk) {
-    set_flag(p.err, CA_FLAG_BOUNDS);
-    cnt = cnt < 0 ? 0 : c.d.nKblk;
-  }
-  int lo = 0, hi = cnt;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (trow[mid] <= last_kb) lo = mid + 1;
-    else hi = mid;
-  }
-  return lo;
-}
 
 // Fused mode: the unit's group table, built by the whole CTA from the
 // bit-packed masks (the Q-block union and intra-group union of the abstract,
@@ -227,9 +152,6 @@ __device__ int fused_group_table(const AttnParams& p, const UnitCoord& uc, int32
   __syncthreads();
   return *total;
 }
-
-// How a piece's result leaves the CTA.
-enum PieceOut : int { kOutFinal = 0, kOutSplit = 1, kOutSK = 2 };
 
 template <int D, int NT, bool QSPLIT, bool KV8>
 __global__ void __launch_bounds__(128 + NT * 128, 1)

@@ -49,10 +49,20 @@ struct AttnParams {
   // E4M3 pages: per table entry (group g, entry e) the (K, V) scales of its
   // page, escale[g * nKblk + e] (built by a gather kernel before the launch)
   const float2* escale;
+  // tile kernel, split tail: units [tail_start, tail_start + n_tail) run as
+  // tail_k pieces each (the last partial wave), leaving fp32 partials that a
+  // merge kernel combines; all earlier units run whole
+  int tail_start, tail_k, n_tail;
+  float* Otail;    // [n_tail * tail_k][128][D]
+  float* LSEtail;  // [n_tail * tail_k][128]
   const SeqDesc* seqs;  // [num_seqs] in device memory, or null: one sequence, seq0
   SeqDesc seq0;
   int num_seqs;
   int Hq, Hkv, G, HPU, nhalves, L, B, num_pages, n_splits, out_f32;  // L = rows of Q / O
+  // order of the units within a sequence: 0 = by query span (later spans, with
+  // more causal blocks, first), 1 = by KV group (all spans of a group together,
+  // so the pages live in L2 at one time are those of few groups)
+  int unit_order;
   float scale_log2;  // log2(e) / sqrt(D)
   unsigned long long wait_ns;
 };
@@ -66,6 +76,11 @@ cudaError_t launch_chunk_attention(const CUtensorMap& q, const CUtensorMap& qlo,
                                    const CUtensorMap& k, const CUtensorMap& v,
                                    const AttnParams& p, int D, int NT, bool qsplit, bool kv8,
                                    int grid, cudaStream_t st);
+// One 128-row tile per CTA, score tile triple-buffered in TMEM (bf16 only);
+// launches the tail merge as well when p.tail_k > 1.
+cudaError_t launch_chunk_attention_tile(const CUtensorMap& q, const CUtensorMap& k,
+                                        const CUtensorMap& v, const AttnParams& p, int D,
+                                        int grid, cudaStream_t st);
 cudaError_t launch_cast_bf16_f16(const void* src, void* dst, size_t n, cudaStream_t st);
 cudaError_t launch_gather_scales(const int32_t* tables, const int32_t* counts,
                                  const int32_t* page_table, const float* K_scale,

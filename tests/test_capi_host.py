@@ -117,12 +117,18 @@ def test_workspace_size_rules(bsc):
     ws = bsc.lib.ca_workspace_size
     # bf16, one CTA per unit: no workspace
     assert ws(0, 32, 8, 128, 64, 2048, 129024, 2048, 1) == 0
-    # automatic mode, 256 units >= 148 SMs: one CTA per unit, no workspace
-    assert ws(0, 32, 8, 128, 64, 2048, 129024, 2048, 0) == 0
-    # automatic mode, 16 units: persistent grid of min(148, 16*12/4) = 48 CTAs,
-    # schedule + fp32 partials of <= 2 pieces per CTA
+    # automatic mode at 128K: 512 one-tile units on 148 SMs; the 68 units of
+    # the last partial wave run as 2 KV pieces each (fp32 partials of 128 rows)
+    tail = 68 * 2 * 128
+    assert ws(0, 32, 8, 128, 64, 2048, 129024, 2048, 0) == tail * 128 * 4 + tail * 4
+    # automatic mode, 2 groups x 2 head pairs x 8 spans = 32 units (< 148 SMs):
+    # every unit in floor(148 / 32) = 4 KV pieces, fp32 partials of every row
     n = ws(0, 8, 2, 128, 64, 512, 1024, 24, 0)
-    assert 2 * 48 * 256 * 128 * 4 <= n < 2 * 48 * 256 * 130 * 4 + 65536
+    assert n == 4 * 512 * 8 * 128 * 4 + 4 * 8 * 512 * 4
+    # fp32 inputs keep the two-tile kernel: its persistent grid of
+    # min(148, 16*12/4) = 48 CTAs with <= 2 partial pieces per CTA
+    n = ws(1, 8, 4, 128, 64, 512, 1024, 24, 0)
+    assert n >= 2 * 48 * 256 * 128 * 4
     # explicit split: fp32 partials + LSE partials
     n = ws(0, 32, 8, 128, 64, 2048, 129024, 2048, 2)
     assert n >= 2 * 2048 * 32 * 128 * 4 + 2 * 32 * 2048 * 4
