@@ -272,6 +272,59 @@ def run_varlen(bsc, dev, stream, reps=12):
             "note": "ca_chunk_attention_varlen, unaligned prefixes and chunk lengths, one launch"}
 
 
+def run_density_sweep(bsc, dev, stream, reps=5):
+    """The 64K density / correlation sweep: prefix 63488 + chunk 2048, 32/8 heads,
+    d 128, bf16, block 64 and 128.  rho is the vertical-slash generator's column
+    density (sink block and 8-block (B 64) or 4-block (B 128) local window on
+    top); rho = 1 is the all-ones mask, once per block size.  Per cell: the
+    attention's device time (mean of `reps` launches after one warm-up), the
+    selected FLOPs, the table density, and the speedup over the same block
+    size's rho = 1 cell.  Page data are seeded device normals, one pool per
+    block size (256 MiB of K and V, more than L2 holds)."""
+    import numpy as np
+    import torch
+
+    import workloads as wl
+    out = {"rho_meaning": "column density of the vertical-slash generator (sink and local "
+                          "window added on top); rho = 1: all-ones mask",
+           "cells": []}
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    for block in (64, 128):
+        w1 = wl.density_cell(1.0, 0.0, block=block)
+        g = torch.Generator(device=dev).manual_seed(block)
+        K = torch.randn(w1.num_pages, w1.Hkv, block, w1.head_dim, generator=g, device=dev).bfloat16()
+        V = torch.randn(w1.num_pages, w1.Hkv, block, w1.head_dim, generator=g, device=dev).bfloat16()
+        Q = torch.randn(w1.chunk_len, w1.Hq, w1.head_dim, generator=g, device=dev).bfloat16()
+        pt = torch.from_numpy(np.random.default_rng(block).permutation(w1.num_pages)
+                              .astype(np.int32)).to(dev)
+        O = torch.empty_like(Q)
+        lse = torch.empty(w1.Hq, w1.chunk_len, dtype=torch.float32, device=dev)
+        n = bsc.workspace_size(torch.bfloat16, w1.Hq, w1.Hkv, w1.head_dim, block, w1.chunk_len,
+                               w1.prefix_len, w1.num_pages)
+        ws = torch.empty(max(n, 1), dtype=torch.uint8, device=dev)
+        cells = [(1.0, 0.0)] + [(r, c) for r in (0.5, 0.2, 0.1, 0.05) for c in (0.0, 0.5, 1.0)]
+        base_ms = None
+        for rho, corr in cells:
+            w = wl.density_cell(rho, corr, block=block)
+            tables, counts = bsc.build_tables(torch.from_numpy(wl.mask_for(w)).to(dev), w.Hkv)
+            run = lambda: bsc.chunk_attention(Q, K, V, pt, tables, counts, w.prefix_len,
+                                              err_flag=err, out=O, lse=lse, workspace=ws)
+            run()
+            ms = statistics.mean(timed_launch(stream, run) for _ in range(reps))
+            flops = bsc.selected_flops(tables.cpu().numpy(), counts.cpu().numpy(), w.Hq, w.nPblk,
+                                       w.nQblk, block, w.head_dim)
+            if base_ms is None:
+                base_ms = ms
+            out["cells"].append({"block": block, "rho": rho, "corr": corr, "ms": ms,
+                                 "tflops": flops / (ms * 1e-3) / 1e12,
+                                 "table_density": float(counts.float().mean().item() / w.nKblk),
+                                 "selected_gflop": flops / 1e9,
+                                 "speedup_vs_rho1": base_ms / ms})
+        bsc.check(err)
+        del K, V
+    return out
+
+
 def timed_launch(stream, fn):
     """Device time (ms) of the launches fn() makes.  A sleep kernel keeps the
     GPU busy while the host enqueues them, so the host-side call overhead of a
@@ -597,6 +650,9 @@ def main():
     # ---- the full chunked-prefill sweep (32 x 4096 tokens), one pass
     sweep_res = run_sweep(bsc, dev, stream)
 
+    # ---- the 64K density / correlation sweep (26 cells)
+    density_res = run_density_sweep(bsc, dev, stream)
+
     # ---- end to end through the public API with pinned host buffers
     chunk_blocks = list(range(w.nPblk, w.nKblk))
     h_mask = torch.from_numpy(wl.mask_for(w, seed=0)).pin_memory()
@@ -708,6 +764,7 @@ def main():
             "speedup_vs_dense": dense_ms_mean / mean_attn,
             "table_build_bits": bits_res,
             "sweep_131k": sweep_res,
+            "density_sweep_64k": density_res,
             "fused_step": fused_res,
             "fp8_kv": fp8_res,
             "varlen_batch": varlen_res,

@@ -133,3 +133,4 @@ __device__ __forceinline__ int unit_live_warp(const AttnParams& p, const UnitCoo
 }
 
 }  // namespace ca
+

@@ -570,7 +570,14 @@ static cudaError_t launch_tile_t(const CUtensorMap& q, const CUtensorMap& k, con
   chunk_attn_tile_kernel<D><<<grid, kTThreads, S::kAlloc, st>>>(q, k, v, p);
   e = cudaGetLastError();
   if (e != cudaSuccess || p.tail_k <= 1 || p.n_tail <= 0) return e;
-  tail_combine_kernel<D><<<dim3(p.n_tail, 128 / 8), 256, 0, st>>>(p);
+  return launch_tail_combine(p, D, st);
+}
+
+cudaError_t launch_tail_combine(const AttnParams& p, int D, cudaStream_t st) {
+  const dim3 grid(p.n_tail, 128 / 8);
+  if (D == 128) tail_combine_kernel<128><<<grid, 256, 0, st>>>(p);
+  else if (D == 64) tail_combine_kernel<64><<<grid, 256, 0, st>>>(p);
+  else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 

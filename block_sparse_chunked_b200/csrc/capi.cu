@@ -65,6 +65,7 @@ struct Plan {
   int G, HPU, NT, nhalves, spb, n_splits;
   int units, persistent, sk_ctas;
   int tile;                          // 1: the one-tile kernel (bf16 pages and Q)
+  int pair;                          // 1: the CTA-pair kernel (bf16, head_dim 128, even units)
   int tail_start, tail_k, n_tail;    // tile kernel: the split last partial wave
 };
 
@@ -87,6 +88,9 @@ bool plan_heads(int Hq, int Hkv, int head_dim, int block, Plan& pl, bool tile = 
     pl.nhalves = (pl.G + pl.HPU - 1) / pl.HPU;
   }
   pl.spb = 128 / block;
+  // CTA pairs take the two head pairs of a group's span together: head_dim
+  // 128 and an even number of head pairs per group (G = 3, 4, 7, 8, ...)
+  pl.pair = (tile && head_dim == 128 && pl.nhalves % 2 == 0) ? 1 : 0;
   pl.tail_start = 0;
   pl.tail_k = 1;
   pl.n_tail = 0;
@@ -108,17 +112,19 @@ bool plan_mode_tile(Plan& pl, long long units, int max_stages, int n_splits, boo
   pl.tail_start = (int)units;
   pl.tail_k = 1;
   pl.n_tail = 0;
-  const long long sms = num_sms();
+  // the pair kernel places a pair of units on a pair of SMs
+  const long long per = pl.pair ? 2 : 1;
+  const long long sms = num_sms() / per, jobs = units / per;
   long long S = n_splits;
   if (S <= 0) {
-    S = units > 0 && units < sms ? std::min<long long>(16, std::max<long long>(1, sms / units)) : 1;
-    const long long r = units % sms;
-    if (exact_units && units >= sms && r > 0) {
+    S = jobs > 0 && jobs < sms ? std::min<long long>(16, std::max<long long>(1, sms / jobs)) : 1;
+    const long long r = jobs % sms;
+    if (exact_units && jobs >= sms && r > 0) {
       const int k = (int)std::min<long long>({4, sms / r, (long long)max_stages});
       if (k >= 2) {
         pl.tail_k = k;
-        pl.n_tail = (int)r;
-        pl.tail_start = (int)(units - r);
+        pl.n_tail = (int)(r * per);
+        pl.tail_start = (int)(units - r * per);
       }
     }
   }
@@ -428,7 +434,9 @@ int run_attention(const char* who, const void* Q, const void* K_pages, const voi
     cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)B, (cuuint64_t)Hkv, (cuuint64_t)num_pages};
     cuuint64_t strides[3] = {(cuuint64_t)D * esz, (cuuint64_t)B * D * esz,
                              (cuuint64_t)Hkv * B * D * esz};
-    cuuint32_t box[4] = {kv8 ? (cuuint32_t)D : 64u, (cuuint32_t)B, 1, 1};
+    // (the pair kernel loads K as 64-row halves of a stage)
+    const cuuint32_t rows = (pl.pair && which == 0) ? 64u : (cuuint32_t)B;
+    cuuint32_t box[4] = {kv8 ? (cuuint32_t)D : 64u, rows, 1, 1};
     cuuint32_t es[4] = {1, 1, 1, 1};
     CUresult r = enc(which ? &tv : &tk,
                      kv8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
@@ -466,7 +474,9 @@ int run_attention(const char* who, const void* Q, const void* K_pages, const voi
   p.out_f32 = dtype == CA_DTYPE_FP32 ? 1 : 0;  // E4M3 pages: O is bf16
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   p.wait_ns = kWaitNs;
-  if (pl.tile)
+  if (pl.pair)
+    e = launch_chunk_attention_pair(tq, tk, tv, p, D, grid, st);
+  else if (pl.tile)
     e = launch_chunk_attention_tile(tq, tk, tv, p, D, grid, st);
   else
     e = launch_chunk_attention(tq, tqlo, tk, tv, p, D, pl.NT, dtype == CA_DTYPE_FP32, kv8, grid,

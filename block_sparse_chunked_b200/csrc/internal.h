@@ -81,6 +81,13 @@ cudaError_t launch_chunk_attention(const CUtensorMap& q, const CUtensorMap& qlo,
 cudaError_t launch_chunk_attention_tile(const CUtensorMap& q, const CUtensorMap& k,
                                         const CUtensorMap& v, const AttnParams& p, int D,
                                         int grid, cudaStream_t st);
+// CTA pairs (cta_group::2 MMAs of M = 256), head_dim 128, an even number of
+// units (two head pairs per span); launches the tail merge as well.
+cudaError_t launch_chunk_attention_pair(const CUtensorMap& q, const CUtensorMap& k,
+                                        const CUtensorMap& v, const AttnParams& p, int D,
+                                        int grid, cudaStream_t st);
+// Merge the KV pieces of the split tail units (one-tile and pair kernels).
+cudaError_t launch_tail_combine(const AttnParams& p, int D, cudaStream_t st);
 cudaError_t launch_cast_bf16_f16(const void* src, void* dst, size_t n, cudaStream_t st);
 cudaError_t launch_gather_scales(const int32_t* tables, const int32_t* counts,
                                  const int32_t* page_table, const float* K_scale,
