@@ -71,8 +71,8 @@ struct PairSmem {  // head_dim 128
   static constexpr int kVOff = kKOff + kPNK * kKSlot;
   static constexpr int kBarOff = kVOff + kPNV * kVSlot;
   // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[3],
-  // p_full[3], pv_done, o_done, drain, xchg[4]
-  static constexpr int kNumBars = 1 + 2 * kPNK + 2 * kPNV + 2 * kPSBufs + 3 + 4;
+  // p_full[3], pv_done[0], o_done, drain, xchg[4], pv_done[1]
+  static constexpr int kNumBars = 1 + 2 * kPNK + 2 * kPNV + 2 * kPSBufs + 3 + 4 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   // row maxima of the two key halves, by stage parity [2][2][128], and the
   // final row sums [2][128]
@@ -137,10 +137,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
   auto v_empty = [&](int s) { return bars + 8u * (1 + 2 * kPNK + kPNV + s); };
   auto s_full = [&](int b) { return bars + 8u * (1 + 2 * kPNK + 2 * kPNV + b); };
   auto p_full = [&](int b) { return bars + 8u * (1 + 2 * kPNK + 2 * kPNV + kPSBufs + b); };
-  const uint32_t pv_done = bars + 8u * (1 + 2 * kPNK + 2 * kPNV + 2 * kPSBufs);
-  const uint32_t o_done = pv_done + 8u;
-  const uint32_t drain = pv_done + 16u;
-  auto xchg = [&](int q) { return pv_done + 24u + 8u * q; };  // halves of a sub-partition's rows
+  const uint32_t pv0 = bars + 8u * (1 + 2 * kPNK + 2 * kPNV + 2 * kPSBufs);
+  const uint32_t o_done = pv0 + 8u;
+  const uint32_t drain = pv0 + 16u;
+  auto xchg = [&](int q) { return pv0 + 24u + 8u * q; };  // halves of a sub-partition's rows
+  // PV(j) completes on pv_done(j % 2).  When the softmax sees S(j) complete,
+  // PV(j-3) has completed too (S(j) was issued after it), so a parity wait for
+  // PV(j-1) on pv_done((j-1) % 2) cannot alias; the softmax waits only at
+  // stages that rescale O.
+  auto pv_done = [&](int j) { return j % 2 == 0 ? pv0 : pv0 + 56u; };
   int* misc = reinterpret_cast<int*>(sm + S::kMiscOff);
   // misc[0] tmem base, [1] live entries, [2] first stage, [3] end stage, [5] abort
   volatile int* abort_flag = misc + 5;
@@ -173,7 +178,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         mbar_init(s_full(b), 1);
         mbar_init(p_full(b), 2 * kPSoftmaxWarps);  // every softmax warp of both CTAs
       }
-      mbar_init(pv_done, 1);
+      mbar_init(pv_done(0), 1);
+      mbar_init(pv_done(1), 1);
       mbar_init(o_done, 1);
       mbar_init(drain, 1);
       for (int q = 0; q < 4; ++q) mbar_init(xchg(q), 64);
@@ -336,7 +342,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
           tc_fence_after();
           issue_pv(j);
           mma_commit_pair_w(v_empty(j % kPNV));
-          mma_commit_pair_w(pv_done);
+          mma_commit_pair_w(pv_done(j));
           const int jn = j + kPSBufs;
           if (jn < n) {
             // S(j+3) reuses buffer b after PV(j) has read P(j) (in-order MMAs)
@@ -463,10 +469,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
       l1 += a1;
       l2 += a2;
       l3 += a3;
-      if (j > 0) {
-        ok = wait_warp(pv_done, (j - 1) & 1, p, abort_flag);
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // O holds the sum over earlier stages at the old max: PV(j-1) must
+        // have finished before this warp's 64 columns of O are rescaled
+        ok = wait_warp(pv_done(j - 1), ((j - 1) >> 1) & 1, p, abort_flag);
         if (!ok) break;
-        if (__any_sync(0xffffffffu, need)) {  // this warp's 64 columns of O
+        {
           tc_fence_after();
           uint32_t r[32];
           for (int c = 0; c < 2; ++c) {
