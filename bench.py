@@ -56,11 +56,15 @@ def load_peaks():
 
 
 def kernel_source_digest(path):
-    """sha256 of a CUDA source with comments and blank lines removed, so that a
-    comment edit does not count as a kernel change."""
+    """sha256 of a CUDA source (and the csrc headers it includes) with comments
+    and blank lines removed, so that a comment edit does not count as a kernel
+    change."""
     import hashlib
     import re
-    text = open(path).read()
+    d = os.path.dirname(path)
+    text = "".join(open(os.path.join(d, f)).read()
+                   for f in [os.path.basename(path), "attn_common.cuh", "ptx.cuh", "internal.h"]
+                   if os.path.exists(os.path.join(d, f)))
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     text = re.sub(r"//[^\n]*", "", text)
     lines = [ln.rstrip() for ln in text.splitlines() if ln.strip()]
@@ -69,11 +73,12 @@ def kernel_source_digest(path):
 
 def load_traffic():
     """DRAM bytes per attention launch from the committed ncu capture
-    (profiles/chunk_attn_kernel_ctx128k_traffic.json), or None when the
+    (profiles/chunk_attn_pair_kernel_ctx128k_traffic.json), or None when the
     kernel source has changed since that capture."""
     try:
-        rec = json.load(open(os.path.join(ROOT, "profiles", "chunk_attn_kernel_ctx128k_traffic.json")))
-        src = os.path.join(ROOT, "block_sparse_chunked_b200", "csrc", "chunk_attention.cu")
+        rec = json.load(open(os.path.join(ROOT, "profiles",
+                                          "chunk_attn_pair_kernel_ctx128k_traffic.json")))
+        src = os.path.join(ROOT, "block_sparse_chunked_b200", "csrc", "attn_pair.cu")
         if kernel_source_digest(src) != rec["source_digest"]:
             return None
         return float(rec["dram_bytes_read"]) + float(rec["dram_bytes_write"])
@@ -773,7 +778,7 @@ def main():
                                     "GB/s": build_gbs, "frac_of_measured_hbm": build_gbs / hbm,
                                     "frac_of_8TBs_nominal": build_gbs / 8000.0,
                                     "saturation": build_sat},
-            "roofline": {"bound": "tensor", "kernel": "chunk_attn_kernel",
+            "roofline": {"bound": "tensor", "kernel": "chunk_attn_pair_kernel",
                          "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": attn_tflops / peak, "peak_source": f"{peak_src} bf16 burst",
                          "frac_of_sustained": attn_tflops / peak_sus,

@@ -78,7 +78,9 @@ struct PairSmem {  // head_dim 128
   // final row sums [2][128]
   static constexpr int kXMaxOff = kMiscOff + 64;
   static constexpr int kXSumOff = kXMaxOff + 2 * 2 * 128 * 4;
-  static constexpr int kBytes = kXSumOff + 2 * 128 * 4;
+  // fused mode: the group's table built in the CTA (entries, union bits, count)
+  static constexpr int kFentOff = kXSumOff + 2 * 128 * 4;
+  static constexpr int kBytes = kFentOff + (kMaxFusedWords * 32 + kMaxFusedWords + 1) * 4;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
@@ -162,6 +164,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
   const int spb = kPStageKeys / p.B;  // pages per stage
   const UnitCoord uc = unit_coord(p, tp.u);
 
+  int32_t* fent = reinterpret_cast<int32_t*>(sm + S::kFentOff);
   if (warp == 8) {
     if (lane == 0) {
       misc[5] = 0;
@@ -182,22 +185,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
       mbar_init(pv_done(1), 1);
       mbar_init(o_done, 1);
       mbar_init(drain, 1);
-      for (int q = 0; q < 4; ++q) mbar_init(xchg(q), 64);
+      for (int q = 0; q < 4; ++q) mbar_init(xchg(q), 2);
       fence_mbar_init();
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
     }
-    const int live = unit_live_warp(p, uc);  // the same for both units of the pair
-    if (lane == 0) {
-      const int nst = (live + spb - 1) / spb;
-      misc[1] = live;
-      misc[2] = (int)((long long)tp.split * nst / tp.nsplit);
-      misc[3] = (int)((long long)(tp.split + 1) * nst / tp.nsplit);
+    if (!p.mask_bits) {
+      const int live = unit_live_warp(p, uc);  // the same for both units of the pair
+      if (lane == 0) {
+        const int nst = (live + spb - 1) / spb;
+        misc[1] = live;
+        misc[2] = (int)((long long)tp.split * nst / tp.nsplit);
+        misc[3] = (int)((long long)(tp.split + 1) * nst / tp.nsplit);
+      }
     }
   } else if (warp == 9) {
     tmem_alloc_pair(sbase + S::kMiscOff, 512);
     tmem_relinquish_pair();
+  }
+  if (p.mask_bits) {
+    // fused mode: the whole CTA builds its group's table from the bit-packed
+    // masks (both CTAs of a pair build the same one); one CTA per group writes
+    // it out
+    const int cnt = fused_group_table(p, uc, fent, kPThreads);
+    if (uc.qs == 0 && uc.hh == 0 && tp.split == 0) {
+      if (p.tables_out) {
+        int32_t* trow_out = p.tables_out + (size_t)uc.g * uc.d.nKblk;
+        for (int e = threadIdx.x; e < uc.d.nKblk; e += kPThreads)
+          trow_out[e] = e < cnt ? fent[e] : -1;
+      }
+      if (threadIdx.x == 0 && p.counts_out) p.counts_out[uc.g] = cnt;
+    }
+    if (threadIdx.x == 0) {
+      const int t_last = min(uc.qs * 64 + 63, uc.d.L - 1);
+      const int last_kb = (uc.d.P + t_last) / p.B;
+      int lo = 0, hi = cnt;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (fent[mid] <= last_kb) lo = mid + 1;
+        else hi = mid;
+      }
+      const int nst = (lo + spb - 1) / spb;
+      misc[1] = lo;
+      misc[2] = (int)((long long)tp.split * nst / tp.nsplit);
+      misc[3] = (int)((long long)(tp.split + 1) * nst / tp.nsplit);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -233,7 +266,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         }
       }
     }
-    const int32_t* trow = table_row(p, uc);
+    const int32_t* trow = p.mask_bits ? fent : table_row(p, uc);
     const int e_begin = s0 * spb, e_end = min(live, s1 * spb);
     int pg_cache = 0, cache_base = -64;
     bool ok = true;
@@ -375,7 +408,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
     const int hl_raw = uc.hh * 2 + sub;
     const bool valid_row = hl_raw < p.G && tl < uc.d.L;
     const int head = uc.g * p.G + min(hl_raw, p.G - 1);
-    const int32_t* trow = table_row(p, uc);
+    const int32_t* trow = p.mask_bits ? fent : table_row(p, uc);
     const int kb_m0 = (uc.d.P + t0) / p.B;
     int mask_e = live;
     while (mask_e > 0 && trow[mask_e - 1] >= kb_m0) --mask_e;
@@ -444,7 +477,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
       // stage, so a fast warp never overwrites a value its partner still reads)
       float* xm = xmax + (j & 1) * 256;
       xm[h * 128 + row] = pmax;
-      mbar_arrive(xchg(q4));  // one phase per stage: 64 arrivals
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xchg(q4));  // one phase per stage: one arrival per warp
       ok = wait_warp(xchg(q4), j & 1, p, abort_flag);
       if (!ok) break;
       const float mx = fmaxf(pmax, xm[(1 - h) * 128 + row]) * sc;
@@ -496,7 +530,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
     float l = lpart;
     if (ok) {
       xsum[h * 128 + row] = lpart;
-      mbar_arrive(xchg(q4));  // phase n
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xchg(q4));  // phase n
       ok = wait_warp(xchg(q4), n & 1, p, abort_flag);
       if (ok) l += xsum[(1 - h) * 128 + row];
     }

@@ -68,8 +68,8 @@ struct TileSmem {
   static constexpr int kVOff = kKOff + kTNK * kKV;
   static constexpr int kBarOff = kVOff + kTNV * kKV;
   // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[3],
-  // p_full[3], pv_done, o_done, drain
-  static constexpr int kNumBars = 1 + 2 * kTNK + 2 * kTNV + 2 * kTSBufs + 3;
+  // p_full[3], pv_done[0], o_done, drain, pv_done[1]
+  static constexpr int kNumBars = 1 + 2 * kTNK + 2 * kTNV + 2 * kTSBufs + 4;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 64;
   static constexpr int kAlloc = kBytes + 1024;            // slack for 1024-byte alignment
@@ -127,9 +127,14 @@ __global__ void __launch_bounds__(kTThreads, 1)
   auto v_empty = [&](int s) { return bars + 8u * (1 + 2 * kTNK + kTNV + s); };
   auto s_full = [&](int b) { return bars + 8u * (1 + 2 * kTNK + 2 * kTNV + b); };
   auto p_full = [&](int b) { return bars + 8u * (1 + 2 * kTNK + 2 * kTNV + kTSBufs + b); };
-  const uint32_t pv_done = bars + 8u * (1 + 2 * kTNK + 2 * kTNV + 2 * kTSBufs);
-  const uint32_t o_done = pv_done + 8u;
-  const uint32_t drain = pv_done + 16u;
+  const uint32_t pv0 = bars + 8u * (1 + 2 * kTNK + 2 * kTNV + 2 * kTSBufs);
+  const uint32_t o_done = pv0 + 8u;
+  const uint32_t drain = pv0 + 16u;
+  // PV(j) completes on pv_done(j % 2).  When the softmax sees S(j) complete,
+  // PV(j-3) has completed too (S(j) was issued after it), so a parity wait for
+  // PV(j-1) on pv_done((j-1) % 2) cannot alias; the softmax waits only at
+  // stages that rescale O.
+  auto pv_done = [&](int j) { return j % 2 == 0 ? pv0 : pv0 + 24u; };
   int* misc = reinterpret_cast<int*>(sm + S::kMiscOff);
   // misc[0] tmem base, [1] live entries, [2] first stage, [3] end stage, [5] abort
   volatile int* abort_flag = misc + 5;
@@ -160,7 +165,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
         mbar_init(s_full(b), 1);
         mbar_init(p_full(b), 4);  // one arrival per softmax warp
       }
-      mbar_init(pv_done, 1);
+      mbar_init(pv_done(0), 1);
+      mbar_init(pv_done(1), 1);
       mbar_init(o_done, 1);
       mbar_init(drain, 1);
       fence_mbar_init();
@@ -308,7 +314,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
         tc_fence_after();
         issue_pv(j);
         mma_commit_w(v_empty(j % kTNV));
-        mma_commit_w(pv_done);
+        mma_commit_w(pv_done(j));
         const int jn = j + kTSBufs;
         if (jn < n) {
           // S(j+3) reuses buffer b: it runs after PV(j) has read P(j) (the
@@ -433,13 +439,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
       l1 += a1;
       l2 += a2;
       l3 += a3;
-      // O holds the sum over earlier stages at the old max.  PV(j-1) must have
-      // finished before O is read or P(j) released (one pv_done phase per
-      // stage, waited in order, so the parity never aliases).
-      if (j > 0) {
-        ok = wait_warp(pv_done, (j - 1) & 1, p, abort_flag);
+      // O holds the sum over earlier stages at the old max: PV(j-1) must have
+      // finished before O is rescaled
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        ok = wait_warp(pv_done(j - 1), ((j - 1) >> 1) & 1, p, abort_flag);
         if (!ok) break;
-        if (__any_sync(0xffffffffu, need)) {
+        {
           tc_fence_after();
           uint32_t r[32];
           for (int c = 0; c < D / 32; ++c) {

@@ -547,8 +547,13 @@ int ca_chunk_attention(const void* Q, const void* K_pages, const void* V_pages, 
 namespace {
 // Fused and E4M3 calls: one CTA per unit (no persistent grid), KV splits when
 // the units do not fill the SMs.
+// pair_ok: the CTA-pair kernel may take the call (bf16, fused tables); it does
+// when its shape rules hold (head_dim 128, an even number of head pairs).
 bool plan_masked(int Hq, int Hkv, int head_dim, int block, int chunk_len, int prefix_len,
-                 int n_splits, Plan& pl, SeqDesc& d, int max_nKblk = 2048) {
+                 int n_splits, Plan& pl, SeqDesc& d, int max_nKblk = 2048, bool pair_ok = false) {
+  if (pair_ok && plan(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl, d, true) &&
+      pl.pair)
+    return d.nKblk <= max_nKblk;
   if (!plan(Hq, Hkv, head_dim, block, chunk_len, prefix_len, 1, pl, d)) return false;
   if (d.nKblk > max_nKblk) return false;
   const int max_stages = (d.nKblk + pl.spb - 1) / pl.spb;
@@ -565,7 +570,8 @@ size_t ca_workspace_size_masked(int dtype, int Hq, int Hkv, int head_dim, int bl
   Plan pl;
   SeqDesc d;
   if (dtype != CA_DTYPE_BF16 && dtype != CA_DTYPE_FP32) return (size_t)-1;
-  if (!plan_masked(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl, d))
+  if (!plan_masked(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl, d, 2048,
+                   dtype == CA_DTYPE_BF16))
     return (size_t)-1;
   if (num_pages < d.nKblk) return (size_t)-1;
   return ws_layout(dtype, Hq, Hkv, head_dim, block, chunk_len, num_pages, pl).total;
@@ -584,7 +590,8 @@ int ca_chunk_attention_masked(const void* Q, const void* K_pages, const void* V_
     return fail(CA_ERR_DTYPE, "%s: dtype code %d not supported", who, dtype);
   Plan pl;
   SeqDesc d;
-  if (!plan_masked(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl, d))
+  if (!plan_masked(Hq, Hkv, head_dim, block, chunk_len, prefix_len, n_splits, pl, d, 2048,
+                   dtype == CA_DTYPE_BF16))
     return fail(CA_ERR_ARG,
                 "%s: unsupported shape Hq=%d Hkv=%d head_dim=%d block=%d chunk_len=%d "
                 "prefix_len=%d (nKblk <= 2048)",
@@ -611,9 +618,10 @@ int ca_chunk_attention_masked(const void* Q, const void* K_pages, const void* V_
   p.counts_out = counts_out;
   p.seq0 = d;
   p.num_seqs = 1;
+  p.unit_order = (pl.tile && (long long)prefix_len >= 2LL * chunk_len) ? 1 : 0;
   return run_attention(who, Q, K_pages, V_pages, dtype, num_pages, Hq, Hkv, head_dim, block,
-                       chunk_len, pl, wl, static_cast<uint8_t*>(workspace),
-                       pl.units * pl.n_splits, p, static_cast<cudaStream_t>(stream));
+                       chunk_len, pl, wl, static_cast<uint8_t*>(workspace), plan_grid(pl), p,
+                       static_cast<cudaStream_t>(stream));
 }
 
 size_t ca_workspace_size_fp8(int Hq, int Hkv, int head_dim, int block, int chunk_len,

@@ -85,74 +85,6 @@ struct Smem {
   static constexpr int kAlloc = kBytes + 1024;          // slack for 1024-B alignment
 };
 
-// Fused mode: the unit's group table, built by the whole CTA from the
-// bit-packed masks (the Q-block union and intra-group union of the abstract,
-// then the compaction) into shared memory: fent[0 .. count) ascending,
-// followed (at fent + 2048) by the group's union bit set (mask_words words)
-// and the count.  Returns the count.
-constexpr int kMaxFusedWords = 64;  // nKblk <= 2048
-__device__ int fused_group_table(const AttnParams& p, const UnitCoord& uc, int32_t* fent,
-                                 int nthreads) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int W = p.mask_words;
-  uint32_t* uni = reinterpret_cast<uint32_t*>(fent + kMaxFusedWords * 32);
-  for (int w = tid; w < W; w += nthreads) uni[w] = 0u;
-  __syncthreads();
-  // OR down the group's G * nQblk rows: thread -> (vector v of a row, rows r,
-  // r + RT, ...), 16-byte loads when the rows allow, several loads in flight
-  const int R = p.G * p.nQblk_mask;
-  const uint32_t* base = p.mask_bits + (size_t)uc.g * R * W;
-  const bool vec4 = (W % 4) == 0 && (reinterpret_cast<uintptr_t>(p.mask_bits) & 15u) == 0;
-  const int NV = vec4 ? W / 4 : W;
-  const int RT = nthreads / NV;
-  if (tid < RT * NV) {
-    const int v = tid % NV;
-    if (vec4) {
-      uint4 acc = make_uint4(0u, 0u, 0u, 0u);
-      const uint4* rowp = reinterpret_cast<const uint4*>(base) + v;
-#pragma unroll 8
-      for (int r = tid / NV; r < R; r += RT) {
-        const uint4 x = __ldg(rowp + (size_t)r * NV);
-        acc.x |= x.x;
-        acc.y |= x.y;
-        acc.z |= x.z;
-        acc.w |= x.w;
-      }
-      if (acc.x) atomicOr(&uni[4 * v], acc.x);
-      if (acc.y) atomicOr(&uni[4 * v + 1], acc.y);
-      if (acc.z) atomicOr(&uni[4 * v + 2], acc.z);
-      if (acc.w) atomicOr(&uni[4 * v + 3], acc.w);
-    } else {
-      uint32_t acc = 0u;
-#pragma unroll 8
-      for (int r = tid / NV; r < R; r += RT) acc |= __ldg(base + (size_t)r * W + v);
-      if (acc) atomicOr(&uni[v], acc);
-    }
-  }
-  __syncthreads();
-  if (tid == 0 && (uc.d.nKblk & 31)) uni[W - 1] &= (1u << (uc.d.nKblk & 31)) - 1u;
-  __syncthreads();
-  // compaction by warp 0: lane l ranks words 2l and 2l + 1
-  int* total = reinterpret_cast<int*>(uni + kMaxFusedWords);
-  if (warp == 0) {
-    const int w0 = 2 * lane;
-    const uint32_t x0 = w0 < W ? uni[w0] : 0u, x1 = w0 + 1 < W ? uni[w0 + 1] : 0u;
-    const int cnt = __popc(x0) + __popc(x1);
-    int incl = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int pos = incl - cnt;
-    for (uint32_t x = x0; x; x &= x - 1) fent[pos++] = w0 * 32 + __ffs(x) - 1;
-    for (uint32_t x = x1; x; x &= x - 1) fent[pos++] = (w0 + 1) * 32 + __ffs(x) - 1;
-    if (lane == 31) *total = incl;
-  }
-  __syncthreads();
-  return *total;
-}
-
 template <int D, int NT, bool QSPLIT, bool KV8>
 __global__ void __launch_bounds__(128 + NT * 128, 1)
     chunk_attn_kernel(const __grid_constant__ CUtensorMap tmQ,

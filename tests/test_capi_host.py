@@ -241,8 +241,13 @@ def test_masked_rejects_bad_arguments(bsc, kw, code):
 
 def test_workspace_size_masked(bsc):
     wm = bsc.lib.ca_workspace_size_masked
-    assert wm(0, 32, 8, 128, 64, 2048, 129024, 2048, 0) == 0           # 256 units: one CTA each
-    assert wm(0, 8, 2, 128, 64, 512, 1024, 24, 0) > 0                  # 16 units: KV splits
+    # bf16, head_dim 128, G = 4: the CTA-pair kernel; at 128K the last partial
+    # wave (68 of 512 units) runs as 2 KV pieces each
+    tail = 68 * 2 * 128
+    assert wm(0, 32, 8, 128, 64, 2048, 129024, 2048, 0) == tail * 128 * 4 + tail * 4
+    assert wm(0, 8, 2, 128, 64, 512, 1024, 24, 0) > 0                  # 32 units: KV splits
+    # fp32 inputs keep the two-tile kernel: 256 units, one CTA each
+    assert wm(1, 32, 8, 128, 64, 2048, 129024, 2048, 0) > 0            # (bf16 copies of Q/K/V)
     assert wm(0, 32, 8, 128, 64, 2048, 129024 + 64, 2049, 0) == ctypes.c_size_t(-1).value
 
 

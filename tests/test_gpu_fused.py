@@ -45,17 +45,20 @@ def compare(O, L, Oo, Lo):
     assert np.abs(O - Oo).max() <= O_TOL
 
 
-def test_fused_bit_identical_to_two_step_128k(bsc):
+@pytest.mark.parametrize("n_splits", [0, 1])
+def test_fused_bit_identical_to_two_step_128k(bsc, n_splits):
+    """Same kernel, same plan (n_splits 0: the last partial wave in KV pieces;
+    1: one CTA per unit), tables built in the CTAs instead of read: bit-identical."""
     w = workloads.get_config("ctx128k")
     x = workloads.make_qkv_pages(w)
     m = workloads.mask_for(w)
-    O, L, t, c = fused(bsc, w, x, m)
+    O, L, t, c = fused(bsc, w, x, m, n_splits=n_splits)
     to, co = oracle.oracle_tables(m, w.Hkv)
     assert np.array_equal(t, to) and np.array_equal(c, co)
     d = {k: v.cuda() for k, v in x.items()}
     tt, cc = bsc.build_tables(torch.from_numpy(m).cuda(), w.Hkv)
     O2, L2 = bsc.chunk_attention(d["Q"], d["K_pages"], d["V_pages"], d["page_table"], tt, cc,
-                                 w.prefix_len, n_splits=1)
+                                 w.prefix_len, n_splits=n_splits)
     assert torch.equal(O, O2) and torch.equal(L, L2)
 
 
