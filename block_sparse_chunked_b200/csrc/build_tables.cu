@@ -10,16 +10,18 @@
 // rows, and the table is the ordered list of nonzero columns.  One thread
 // block cluster (up to 8 CTAs) owns one (mask, group): each CTA reduces a
 // column slab with 16-, 4- or 1-byte loads, turns it into a bit set in shared
-// memory, and compacts it with per-word popcounts and a block scan; the CTAs
-// exchange their slab counts through distributed shared memory to place
-// their entries.  No global scratch, no atomics on global memory, and the
-// output is deterministic.  HBM-bound: every mask byte is read exactly once.
+// memory, and compacts it with per-word popcounts and a block scan; each CTA
+// stores its slab count into the shared memory of every CTA of its cluster
+// (one cluster barrier), then places its entries.  No global scratch, no
+// atomics on global memory, and the output is deterministic.  HBM-bound:
+// every mask byte is read exactly once.
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -30,6 +32,9 @@ namespace ca {
 #endif
 #ifndef CA_BUILD_UNROLL
 #define CA_BUILD_UNROLL 8
+#endif
+#ifndef CA_BUILD_MIN_BLOCKS
+#define CA_BUILD_MIN_BLOCKS 4
 #endif
 constexpr int kBuildThreads = 256;
 constexpr int kRowUnroll = CA_BUILD_UNROLL;
@@ -80,15 +85,20 @@ struct VecLoad<1> {
 
 // grid = (C, Hkv, nb), cluster = (C, 1, 1); slab = columns per CTA (multiple of 32).
 template <int VEC>
-__global__ void __launch_bounds__(kBuildThreads)
+__global__ void __launch_bounds__(kBuildThreads, CA_BUILD_MIN_BLOCKS)
     build_tables_kernel(const uint8_t* __restrict__ mask, int Hq, int Hkv, int nQblk, int nKblk,
                         int slab, int32_t* __restrict__ tables, int32_t* __restrict__ counts) {
   using V = VecLoad<VEC>;
   using T = typename V::T;
   __shared__ uint32_t bits[kMaxSlab / 32];
+  __shared__ int word_off[kMaxSlab / 32];  // entries of the slab before word w
   __shared__ int warp_sum[kBuildThreads / 32];
-  __shared__ int slab_total;
+  __shared__ int slab_count[8];  // [r]: set columns in the slab of cluster rank r
 
+  // Phase 0 of the cluster barrier: this CTA is running.  Its wait (after the
+  // loads) guarantees that every CTA of the cluster has started before any
+  // CTA stores into another's shared memory.
+  cluster_arrive_relaxed();
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
   const int C = (int)cluster.num_blocks();
@@ -151,34 +161,33 @@ __global__ void __launch_bounds__(kBuildThreads)
     wbase += (w < warp) ? warp_sum[w] : 0;
     tot += warp_sum[w];
   }
-  const int excl = wbase + incl - cnt;
-  if (tid == 0) slab_total = tot;
+  if (tid < nwords) word_off[tid] = wbase + incl - cnt;
 
-  // ---- cluster: offsets of this slab and the group's total through DSMEM.
-  cluster.sync();
+  // ---- cluster: every CTA learns every slab count.  Rank r's count goes to
+  // slab_count[r] of each CTA; after the barrier all reads are local, so no
+  // CTA touches another's shared memory once it may have exited.
+  cluster_wait_acquire();
+  if (tid < C) st_cluster_s32(mapa_rank(smem_u32(&slab_count[rank]), (uint32_t)tid), tot);
+  cluster_arrive_release();
+  cluster_wait_acquire();
   int before = 0, total = 0;
   for (int r = 0; r < C; ++r) {
-    const int t = *cluster.map_shared_rank(&slab_total, r);
+    const int t = slab_count[r];
     before += (r < rank) ? t : 0;
     total += t;
   }
 
   int32_t* trow = tables + ((size_t)b * Hkv + g) * nKblk;
-  // Each warp writes the entries of its 32 words: for word j, lane l handles
-  // column 32j+l; its position is the word's offset plus the set bits below l.
-  for (int j = 0; j < 32; ++j) {
-    const uint32_t wj = __shfl_sync(0xffffffffu, word, j);
-    const int oj = __shfl_sync(0xffffffffu, excl, j);
-    if (wj == 0u) continue;
-    if ((wj >> lane) & 1u) {
-      const int pos = before + oj + __popc(wj & ((1u << lane) - 1u));
-      trow[pos] = c0 + (warp * 32 + j) * 32 + lane;
-    }
+  // Word w is written by warp w % 8: lane l handles column 32w + l, at the
+  // word's offset plus the set bits below l.
+  for (int w = warp; w < nwords; w += kBuildThreads / 32) {
+    const uint32_t x = bits[w];
+    if ((x >> lane) & 1u)
+      trow[before + word_off[w] + __popc(x & ((1u << lane) - 1u))] = c0 + w * 32 + lane;
   }
   // -1 padding of the positions [total, nKblk) that fall inside this slab.
   for (int p = max(total, c0) + tid; p < c1; p += kBuildThreads) trow[p] = -1;
   if (rank == 0 && tid == 0) counts[(size_t)b * Hkv + g] = total;
-  cluster.sync();  // keep slab_total alive until every CTA has read it
 }
 
 template __global__ void build_tables_kernel<16>(const uint8_t*, int, int, int, int, int,

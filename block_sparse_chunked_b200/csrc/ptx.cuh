@@ -309,6 +309,26 @@ __device__ __forceinline__ void cluster_sync_all() {
                    : "memory");
 }
 
+// The two halves of a cluster barrier, for a CTA that has work to do between
+// them.  arrive_relaxed orders no memory (used at kernel start, to say "this
+// CTA is running"); arrive_release makes this thread's earlier writes,
+// shared::cluster stores to other CTAs included, visible to every thread that
+// returns from the matching wait_acquire.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Store a 32-bit value at a shared::cluster address (any CTA of the cluster).
+__device__ __forceinline__ void st_cluster_s32(uint32_t addr, int32_t v) {
+  asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 // The shared::cluster address of the same offset in the CTA of rank `rank`.
 __device__ __forceinline__ uint32_t mapa_rank(uint32_t local, uint32_t rank) {
   uint32_t r;
