@@ -222,16 +222,25 @@ def run_sweep(bsc, dev, stream, n_chunks=32):
             "per_chunk_ms_first_last": [method_ms[0], method_ms[-1]]}
 
 
-def run_varlen(bsc, dev, stream, reps=12):
-    """A batch of 8 sequences with unaligned prefixes and chunk lengths over one
+# The bench's two batches: 8 sequences of long unaligned chunks (many units),
+# and 4 short chunks over long prefixes (9 query spans x 8 groups x 2 head
+# pairs = 144 units, fewer than the SMs).
+VARLEN_LONG = [(121037, 2048), (64005, 1500), (32868, 1024), (100063, 777), (8000, 512),
+               (120001, 2000), (50030, 1900), (90011, 1100)]
+VARLEN_SHORT = [(121037, 192), (64005, 128), (32868, 160), (100063, 64)]
+
+
+def run_varlen(bsc, dev, stream, seqs=VARLEN_LONG, n_splits=1, reps=12,
+               note="ca_chunk_attention_varlen, unaligned prefixes and chunk lengths, one launch"):
+    """A batch of sequences with unaligned prefixes and chunk lengths over one
     shuffled page pool, through one ca_chunk_attention_varlen launch (tables
-    built per sequence beforehand).  Seeded device data; 32/8 heads, d 128."""
+    built per sequence beforehand).  Seeded device data; 32/8 heads, d 128.
+    Times lone launches (behind a sleep kernel) and, for the same work, eight
+    launches back to back between one pair of events."""
     import numpy as np
     import torch
 
     import workloads as wl
-    seqs = [(121037, 2048), (64005, 1500), (32868, 1024), (100063, 777), (8000, 512),
-            (120001, 2000), (50030, 1900), (90011, 1100)]
     Hq, Hkv, d, B = 32, 8, 128, 64
     nKs = [-(-(P + L) // B) for P, L in seqs]
     num_pages = sum(nKs)
@@ -261,20 +270,25 @@ def run_varlen(bsc, dev, stream, reps=12):
     O = torch.empty_like(Q)
     lse = torch.empty(Hq, total_q, dtype=torch.float32, device=dev)
     max_kv = max(P + L for P, L in seqs)
-    n = bsc.lib.ca_workspace_size_varlen(0, Hq, Hkv, d, B, len(seqs), total_q, max_kv, num_pages, 1)
+    n = bsc.lib.ca_workspace_size_varlen(0, Hq, Hkv, d, B, len(seqs), total_q, max_kv, num_pages,
+                                         n_splits)
     ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    call = lambda: bsc.chunk_attention_varlen(  # noqa: E731
+        Q, K, V, cu_q, prefix, pt, cu_pages, flat, counts, max_kv, n_splits=n_splits,
+        err_flag=err, out=O, lse=lse, workspace=ws)
     ts = []
     for r in range(reps):
-        t_ = timed_launch(stream, lambda: bsc.chunk_attention_varlen(
-            Q, K, V, cu_q, prefix, pt, cu_pages, flat, counts, max_kv, n_splits=1, err_flag=err,
-            out=O, lse=lse, workspace=ws))
+        t_ = timed_launch(stream, call)
         if r >= 3:
             ts.append(t_)
+    b2b = timed_launch(stream, lambda: [call() for _ in range(8)]) / 8
     bsc.check(err)
     ms = sum(ts) / len(ts)
+    units = sum(-(-L // 64) for _, L in seqs) * Hkv * ((Hq // Hkv + 1) // 2)
     return {"sequences": len(seqs), "query_tokens": total_q, "kv_tokens": sum(P + L for P, L in seqs),
-            "ms": ms, "selected_gflop": flops / 1e9, "tflops": flops / (ms * 1e-3) / 1e12,
-            "note": "ca_chunk_attention_varlen, unaligned prefixes and chunk lengths, one launch"}
+            "units": units, "n_splits": n_splits, "ms": ms, "selected_gflop": flops / 1e9,
+            "tflops": flops / (ms * 1e-3) / 1e12, "back_to_back_ms": b2b,
+            "back_to_back_tflops": flops / (b2b * 1e-3) / 1e12, "note": note}
 
 
 def run_density_sweep(bsc, dev, stream, reps=5):
@@ -571,6 +585,19 @@ def main():
         bt.append(timed_launch(stream, lambda: bsc.build_tables_batched(mb[r % 4], w.Hkv, tb, cb)))
     bbytes = bsc.builder_bytes(nb, w.Hq, w.Hkv, w.nQblk, w.nKblk)
     build_gbs = bbytes / (statistics.mean(bt) * 1e-3) / 1e9
+    # the same 12 launches back to back between one pair of events (each set
+    # was last read three launches, 207 MB, earlier), and the floor a lone
+    # launch pays under this event method: an empty kernel timed the same way
+    a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(200_000)
+    a_.record(stream)
+    for r in range(12):
+        bsc.build_tables_batched(mb[r % 4], w.Hkv, tb, cb)
+    b_.record(stream)
+    torch.cuda.synchronize()
+    b2b_us = a_.elapsed_time(b_) * 1e3 / 12
+    floor_us = statistics.mean(timed_launch(stream, lambda: torch.cuda._sleep(0))
+                               for _ in range(8)) * 1e3
     # saturation: the four batches as one launch of 128 masks (277 MB, more than L2 holds)
     mb_all = torch.cat(mb)
     tb_all = torch.empty(4 * nb, w.Hkv, w.nKblk, dtype=torch.int32, device=dev)
@@ -645,12 +672,25 @@ def main():
     fp8_res = {"ms": statistics.mean(fp8_ms),
                "tflops": mean_flops / (statistics.mean(fp8_ms) * 1e-3) / 1e12,
                "kv_cache_bytes": 2 * K8.numel(), "bf16_kv_cache_bytes": 4 * K8.numel(),
+               "role": "memory-capacity option: half the KV cache bytes, not a speed-up",
+               "vs_bf16_time": statistics.mean(fp8_ms) / mean_attn,
+               "why_slower": "the MMAs need f16 operands (an 8-bit MMA would need Q and P in "
+                             "8 bits, ~2^-4 score error); two warps widen each stage's E4M3 "
+                             "bytes to f16 in shared memory, which doubles the kernel's "
+                             "instructions and runs on the two-tile kernel",
                "note": "ca_chunk_attention_fp8 incl. the Q cast and scale gather; one page "
                        "buffer (not rotated)"}
     del K8, V8
 
     # ---- a batch of sequences with unaligned lengths (one varlen launch)
     varlen_res = run_varlen(bsc, dev, stream)
+    varlen_short = {
+        "auto": run_varlen(bsc, dev, stream, VARLEN_SHORT, n_splits=0,
+                           note="ca_chunk_attention_varlen, 4 short chunks over long prefixes, "
+                                "automatic plan"),
+        "one_cta_per_unit": run_varlen(bsc, dev, stream, VARLEN_SHORT, n_splits=1,
+                                       note="the same batch, n_splits = 1"),
+    }
 
     # ---- the full chunked-prefill sweep (32 x 4096 tokens), one pass
     sweep_res = run_sweep(bsc, dev, stream)
@@ -773,10 +813,18 @@ def main():
             "fused_step": fused_res,
             "fp8_kv": fp8_res,
             "varlen_batch": varlen_res,
+            "varlen_short_batch": varlen_short | {
+                "vs_single_sequence": varlen_short["auto"]["tflops"] / attn_tflops,
+                "vs_single_sequence_back_to_back":
+                    varlen_short["auto"]["back_to_back_tflops"] / attn_tflops},
             "kv_append": append_res,
             "table_build_batched": {"masks_per_launch": nb, "us": statistics.mean(bt) * 1e3,
                                     "GB/s": build_gbs, "frac_of_measured_hbm": build_gbs / hbm,
                                     "frac_of_8TBs_nominal": build_gbs / 8000.0,
+                                    "back_to_back_us": b2b_us,
+                                    "back_to_back_frac_of_measured_hbm":
+                                        bbytes / (b2b_us * 1e-6) / 1e9 / hbm,
+                                    "empty_launch_floor_us": floor_us,
                                     "saturation": build_sat},
             "roofline": {"bound": "tensor", "kernel": "chunk_attn_pair_kernel",
                          "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",

@@ -135,12 +135,15 @@ size_t ca_workspace_size(int dtype, int Hq, int Hkv, int head_dim, int block, in
  *   O           [L, Hq, d] (out), dtype `dtype`
  *   LSE         float32 [Hq, L] (out), natural log
  *   workspace   >= ca_workspace_size(...) bytes (may be NULL if that is 0)
- *   n_splits    <= 0: automatic — one CTA per unit when there are at least
- *               as many units (group x 64-token span x head slice) as SMs;
- *               otherwise a persistent grid of at most one CTA per SM splits
- *               all units' KV stages evenly and merges the pieces of split
- *               units by LSE (needs workspace); 1: one CTA per unit; k > 1:
- *               each unit's KV range split k ways, merged by LSE
+ *   n_splits    <= 0: automatic.  bf16: with fewer units (group x 64-token
+ *               span x head slice) than SMs, each unit's KV range is split
+ *               into floor(SMs / units) pieces (at most 16); otherwise one
+ *               CTA per unit, and the units of the last partial wave run as
+ *               up to 4 pieces each.  fp32 / E4M3: one CTA per unit when the
+ *               units fill the SMs, else a persistent grid of at most one
+ *               CTA per SM that splits all units' KV stages evenly.  Pieces
+ *               are merged by LSE (needs workspace).  1: one CTA per unit;
+ *               k > 1: each unit's KV range split k ways, merged by LSE
  *   err_flag    int32 (device, may be NULL): the kernels OR CA_FLAG_* into it
  *               on an out-of-range table entry / page id (the access is
  *               clamped, results are then undefined) or on a pipeline wait
@@ -186,8 +189,14 @@ size_t ca_workspace_size_varlen(int dtype, int Hq, int Hkv, int head_dim, int bl
  *               cu_pages[s+1] - cu_pages[s] >= nKblk_s
  *   max_kv_len  host bound on P_s + L_s (sizes KV splits)
  *   workspace   >= ca_workspace_size_varlen(...) bytes (never NULL)
- *   n_splits    <= 0 or 1: one CTA per (sequence, group, span, head slice);
- *               k > 1: KV range split k ways, merged by LSE
+ *   n_splits    1: one CTA per unit (sequence, group, 64-token span, head
+ *               slice); <= 0: automatic — bf16: when the batch's unit bound
+ *               ((ceil(total_q / 64) + num_seqs) x Hkv x head slices) is
+ *               below the SM count, each unit's KV range in
+ *               floor(SMs / bound) pieces (at most 16, at most
+ *               ceil(max_kv_len / 128)), else one CTA per unit; fp32: one
+ *               CTA per unit; k > 1: KV range split k ways; pieces merged by
+ *               LSE
  * Everything runs on the stream from device arrays (capturable in a CUDA
  * graph).  A sequence whose offsets are inconsistent is skipped (its rows
  * are left unwritten) and CA_FLAG_BOUNDS is set in *err_flag.

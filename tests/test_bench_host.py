@@ -29,8 +29,9 @@ def test_digest_ignores_comments(tmp_path):
 def test_traffic_reported_only_for_the_captured_kernel():
     import json
     b = _bench()
-    rec = json.load(open(os.path.join(ROOT, "profiles", "chunk_attn_kernel_ctx128k_traffic.json")))
-    src = os.path.join(ROOT, "block_sparse_chunked_b200", "csrc", "chunk_attention.cu")
+    rec = json.load(open(os.path.join(ROOT, "profiles",
+                                      "chunk_attn_pair_kernel_ctx128k_traffic.json")))
+    src = os.path.join(ROOT, "block_sparse_chunked_b200", "csrc", "attn_pair.cu")
     same = b.kernel_source_digest(src) == rec["source_digest"]
     t = b.load_traffic()
     if same:

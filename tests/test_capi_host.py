@@ -288,3 +288,4 @@ def test_accounting_general_lengths_match_aligned(bsc):
             last_tok = min(qb * B + B - 1, L - 1)
             brute += sum(1 for e in t[g, :c[g]] if e * B <= P + last_tok)
     assert bsc.selected_pairs_pl(t, c, Hq, P, L, B) == brute
+

@@ -127,13 +127,32 @@ BATCHES = [
 
 
 @pytest.mark.parametrize("bi", range(len(BATCHES)))
-@pytest.mark.parametrize("n_splits", [1, 2])
+@pytest.mark.parametrize("n_splits", [0, 1, 2])
 def test_varlen_batch(bsc, bi, n_splits):
     b = make_batch(BATCHES[bi], seed=bi)
     O, L, flat, counts, err = run_batch(bsc, b, n_splits)
     bsc.check(err)
     Oo, Lo = batch_oracle(b, flat, counts)
     compare(O.float().cpu().numpy(), L.cpu().numpy(), Oo, Lo)
+
+
+# Short chunks over long prefixes: fewer units than SMs (the automatic plan
+# splits every unit's KV range when the batch's unit bound is below the SM
+# count).  The last sequence has one token.
+SHORT = [(30000, 64), (9000, 100), (15000, 37), (20000, 128), (2000, 1)]
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_varlen_short_batch(bsc, d):
+    b = make_batch(SHORT, d=d, seed=11)
+    O, L, flat, counts, err = run_batch(bsc, b, n_splits=0)
+    bsc.check(err)
+    Oo, Lo = batch_oracle(b, flat, counts)
+    compare(O.float().cpu().numpy(), L.cpu().numpy(), Oo, Lo)
+    # the split pieces are merged in a fixed order: the same bits every run
+    O2, L2, _, _, err2 = run_batch(bsc, b, n_splits=0)
+    bsc.check(err2)
+    assert torch.equal(O, O2) and torch.equal(L, L2)
 
 
 def test_varlen_short_page_span_is_flagged(bsc):
