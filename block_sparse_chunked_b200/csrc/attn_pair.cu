@@ -353,7 +353,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           if (kk < nk)
-            mma_ts_pair_w(tmem, at + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), kIdescPV,
+            mma_ts_pair_w(tmem, at + (kk & 3) * 8 + (kk >> 2) * 64,
+                          vd + (uint64_t)((kk * 16 * 128) >> 4), kIdescPV,
                           kk > 0 ? 1u : acc0);
       };
       bool ok = true;
@@ -445,7 +446,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         }
       }
       // exponentiate this half against the running max while taking its max;
-      // P (bf16 pairs) goes to TMEM columns [32 h, 32 h + 32) of the buffer
+      // P (bf16 pairs) goes to TMEM columns [64 h, 64 h + 32) of the buffer:
+      // inside this warp's own half of S, which the other warp of the row
+      // never reads (PV takes keys 64 .. 127 from column 64)
       const float sc = p.scale_log2;
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
       auto pass = [&](float nm, bool with_max) {
@@ -468,7 +471,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
             else fadd2(a0, a1, e0, e1);
             pk[i] = pack_bf16x2(e0, e1);
           }
-          tmem_st16(tS + h * (kHalf / 2) + c * 16, pk);
+          tmem_st16(tS + h * kHalf + c * 16, pk);
         }
         return fmaxf(mx0, mx1);
       };
