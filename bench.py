@@ -87,7 +87,9 @@ def load_traffic():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms during the timed
+    region; the SM clock is the median of the samples under load (power draw in
+    the upper half of the range seen, all samples if the range is flat)."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -101,7 +103,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -138,9 +140,13 @@ class ClockSampler:
                     reasons.add(n)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "samples": len(sm), "power_w_max": max(power) if power else None,
-                "reasons": sorted(reasons)}
+        loaded = sm
+        if len(power) == len(sm) and max(power) - min(power) > 20.0:
+            cut = (max(power) + min(power)) / 2
+            loaded = [c for c, w in zip(sm, power) if w >= cut]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "samples": len(sm), "samples_under_load": len(loaded),
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
 
 
 def max_over_ranks(values, dist=None, device=None):
@@ -417,7 +423,12 @@ def reference_arm(args, rank):
     mask = workloads.mask_for(w, seed=0)
     for _ in range(args.warmup):
         cpu_oracle_sample(w, x, mask, stride=256)
-    res = [cpu_oracle_sample(w, x, mask, stride=64) for _ in range(args.steps)]
+    # every 64th token per step up to 150 steps, then a sparser sample per step
+    # (the stride doubles), so that K steps stay around a minute of host time
+    stride = 64
+    while stride < w.chunk_len and args.steps > 150 * (stride // 64):
+        stride *= 2
+    res = [cpu_oracle_sample(w, x, mask, stride=stride) for _ in range(args.steps)]
     v = statistics.mean(r["value"] for r in res)
     secs = statistics.mean(r["seconds"] for r in res)
     line = {
@@ -435,7 +446,7 @@ def reference_arm(args, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -535,11 +546,9 @@ def main():
     step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(args.steps)]
     build_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
     attn_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
-    flops = []
-    for i in range(args.steps):
-        s = sets[i % len(sets)]
-        flops.append(bsc.selected_flops(s["tables"].cpu().numpy(), s["counts"].cpu().numpy(),
-                                        w.Hq, w.nPblk, w.nQblk, w.block, w.head_dim))
+    set_flops = [bsc.selected_flops(s["tables"].cpu().numpy(), s["counts"].cpu().numpy(),
+                                    w.Hq, w.nPblk, w.nQblk, w.block, w.head_dim) for s in sets]
+    flops = [set_flops[i % len(sets)] for i in range(args.steps)]
     mean_step = statistics.mean(step_ms)
     mean_attn = statistics.mean(attn_ms)
     mean_flops = statistics.mean(flops)

@@ -78,8 +78,9 @@ def test_density_grid_cell(bsc, rho, corr, block):
     t, c = tables.cpu().numpy(), counts.cpu().numpy()
     to, co = oracle.oracle_tables(m, w.Hkv)
     assert np.array_equal(t, to) and np.array_equal(c, co), "tables differ from the oracle"
-    if rho >= 1.0:
+    if rho >= 1.0:  # the all-ones cell: exactly the density-100% path's tables
         assert c.tolist() == [w.nKblk] * w.Hkv
+        assert np.array_equal(t, np.tile(np.arange(w.nKblk, dtype=t.dtype), (w.Hkv, 1)))
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     O, L = bsc.chunk_attention(d["Q"], d["K_pages"], d["V_pages"], d["page_table"], tables,
                                counts, w.prefix_len, err_flag=err)
