@@ -15,9 +15,13 @@ __device__ __forceinline__ void set_flag(int32_t* err, int f) {
 }
 
 // Warp-uniform bounded wait.  Returns false (and flags / aborts) on expiry.
+// A phase that has already completed is taken without reading the abort flag
+// (its data is ready either way); only a wait that would block first checks
+// whether another warp has given up.
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, const AttnParams& p,
                                           volatile int* abort_flag) {
-  bool ok = (*abort_flag == 0) && mbar_wait(bar, parity, p.wait_ns);
+  bool ok = mbar_try_wait(bar, parity) ||
+            ((*abort_flag == 0) && mbar_wait(bar, parity, p.wait_ns));
   ok = __all_sync(0xffffffffu, ok);
   if (!ok) {
     if ((threadIdx.x & 31) == 0 && *abort_flag == 0) {

@@ -488,7 +488,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
       const float m_new = fmaxf(m_used, mx);
       const bool need = (m_new != -INFINITY) && (m_new > m_used + 8.0f);
       float alpha = 1.f;
-      if (__any_sync(0xffffffffu, need)) {  // both halves decide alike
+      const bool redo = __any_sync(0xffffffffu, need);
+      if (redo) {  // both halves decide alike
         if (need) {
           alpha = ex2(m_used - m_new);
           l0 *= alpha;
@@ -506,7 +507,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
       l1 += a1;
       l2 += a2;
       l3 += a3;
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
+      if (j > 0 && redo) {
         // O holds the sum over earlier stages at the old max: PV(j-1) must
         // have finished before this warp's 64 columns of O are rescaled
         ok = wait_warp(pv_done(j - 1), ((j - 1) >> 1) & 1, p, abort_flag);

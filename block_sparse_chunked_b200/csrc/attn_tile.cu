@@ -423,7 +423,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
       const float m_new = fmaxf(m_used, mx);
       const bool need = (m_new != -INFINITY) && (m_new > m_used + 8.0f);
       float alpha = 1.f;
-      if (__any_sync(0xffffffffu, need)) {
+      const bool redo = __any_sync(0xffffffffu, need);
+      if (redo) {
         if (need) {
           alpha = ex2(m_used - m_new);  // 0 when m_used == -inf
           l0 *= alpha;
@@ -441,7 +442,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
       l3 += a3;
       // O holds the sum over earlier stages at the old max: PV(j-1) must have
       // finished before O is rescaled
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
+      if (j > 0 && redo) {
         ok = wait_warp(pv_done(j - 1), ((j - 1) >> 1) & 1, p, abort_flag);
         if (!ok) break;
         {
