@@ -445,27 +445,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
           }
         }
       }
-      // exponentiate this half against the running max while taking its max;
-      // P (bf16 pairs) goes to TMEM columns [64 h, 64 h + 32) of the buffer:
-      // inside this warp's own half of S, which the other warp of the row
-      // never reads (PV takes keys 64 .. 127 from column 64)
+      // exponentiate this half against the running max; P (bf16 pairs) goes
+      // to TMEM columns [64 h, 64 h + 32) of the buffer: inside this warp's
+      // own half of S, which the other warp of the row never reads (PV takes
+      // keys 64 .. 127 from column 64)
       const float sc = p.scale_log2;
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-      auto pass = [&](float nm, bool with_max) {
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+      auto pass = [&](float nm) {
         a0 = a1 = a2 = a3 = 0.f;
 #pragma unroll
         for (int c = 0; c < kHalf / 32; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float s0v = sr[c * 32 + 2 * i], s1v = sr[c * 32 + 2 * i + 1];
-            if (with_max) {
-              if (i & 1) mx1 = max3(mx1, s0v, s1v);
-              else mx0 = max3(mx0, s0v, s1v);
-            }
             float x0, x1;
-            ffma2(x0, x1, s0v, s1v, sc, sc, nm, nm);
+            ffma2(x0, x1, sr[c * 32 + 2 * i], sr[c * 32 + 2 * i + 1], sc, sc, nm, nm);
             const float e0 = ex2(x0), e1 = ex2(x1);
             if (i & 1) fadd2(a2, a3, e0, e1);
             else fadd2(a0, a1, e0, e1);
@@ -473,9 +467,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
           }
           tmem_st16(tS + h * kHalf + c * 16, pk);
         }
-        return fmaxf(mx0, mx1);
       };
-      const float pmax = mine ? pass(m_used == -INFINITY ? 0.f : -m_used, true) : -INFINITY;
+      // The max of the half is needed only if it may exceed m_used + 8, i.e.
+      // if some exponential exceeds 2^8: never while the sum of the half's
+      // (positive) exponentials stays <= 256, and always before the row has
+      // a max.  Otherwise the half cannot move the max and reports -inf.
+      float pmax = -INFINITY;
+      if (mine) {
+        pass(m_used == -INFINITY ? 0.f : -m_used);
+        const float asum = (a0 + a1) + (a2 + a3);
+        const bool big = !(asum <= 256.f) || m_used == -INFINITY;
+        if (__any_sync(0xffffffffu, big)) {
+          float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < kHalf / 2; ++i) {
+            if (i & 1) mx1 = max3(mx1, sr[2 * i], sr[2 * i + 1]);
+            else mx0 = max3(mx0, sr[2 * i], sr[2 * i + 1]);
+          }
+          pmax = fmaxf(mx0, mx1);
+        }
+      }
       // the row's max: both halves, through shared memory (slots alternate by
       // stage, so a fast warp never overwrites a value its partner still reads)
       float* xm = xmax + (j & 1) * 256;
@@ -500,7 +511,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         }
         if (mine) {
           tmem_wait_st();
-          pass(m_used == -INFINITY ? 0.f : -m_used, false);
+          pass(m_used == -INFINITY ? 0.f : -m_used);
         }
       }
       l0 += a0;
