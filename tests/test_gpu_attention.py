@@ -109,6 +109,31 @@ def test_odd_table_lengths_use_half_stage(bsc):
     compare(O, Lg, *full_oracle(w, x, t, c))
 
 
+@pytest.mark.parametrize("d", [128, 64])
+@pytest.mark.parametrize("n_splits", [0, 3])
+def test_row_max_jumps_mid_row(bsc, d, n_splits):
+    """The running max of the rows jumps by more than 2^8 (log2 units) at
+    three later stages, in either key half of a 128-key stage, so the stage
+    is redone and O rescaled mid-row.  Every query leans on coordinate 0
+    (+4); the keys of prefix blocks 4, 7 and 10 are lam * e_0, with q.k /
+    sqrt(d) = (q_0 + 4) * (10, 25, 40) / 4 against O(1) for the other keys."""
+    w = workloads.Workload("jump", 8, 2, d, "bf16", 1024, 256, 64, "ones", rho=1.0)
+    x = workloads.make_qkv_pages(w)
+    Q = x["Q"].float()
+    Q[..., 0] += 4.0
+    K = x["K_pages"].float()
+    pt = x["page_table"].numpy()
+    for kb, target in ((4, 10.0), (7, 25.0), (10, 40.0)):
+        K[pt[kb]] = 0.0
+        K[pt[kb], :, :, 0] = target * d ** 0.5 / 4.0
+    x = dict(x, Q=Q.to(torch.bfloat16), K_pages=K.to(torch.bfloat16))
+    m = workloads.mask_for(w)
+    O, Lg, t, c = gpu_run(bsc, w, x, m, n_splits=n_splits)
+    Oo, Lo = full_oracle(w, x, t, c)
+    assert np.isfinite(Lo).all() and (Lo > 20.0).mean() > 0.9  # the spikes dominate the rows
+    compare(O, Lg, Oo, Lo)
+
+
 def test_diagonal_missing_and_future_blocks(bsc):
     """No diagonal block selected, plus blocks above the causal diagonal (unclipped)."""
     w = workloads.Workload("nodiag", 8, 2, 128, "bf16", 512, 256, 64, "bernoulli", rho=0.2)
